@@ -1,0 +1,26 @@
+"""fp64 CPU oracle for bipartite prefix-shared attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py`` (its ``cpu_baseline`` leg and its ``--impl reference`` arm) may
+import, call or execute anything in this package.  The CUDA library and its
+Python binding never import it, and the oracle imports nothing from them: the
+two share no code.  Inputs for both come from the separate ``workloads``
+generator module.
+
+What it computes is the plain definition of the operation, written out with
+no blocking, fusion or reordering beyond what the definition states; see
+``oracle.attention`` for the definition and the readings it rests on.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(brute force, closed forms, the four invariants, a library routine); none is
+"parity unpinned".
+"""
+
+from .attention import (  # noqa: F401
+    attend,
+    request_keys,
+    bipartite_attention,
+    bipartite_attention_split,
+    merge_partials,
+    chunk_partial,
+)
