@@ -1,0 +1,168 @@
+/*
+ * bat.h - C ABI of libbat.so: bipartite prefix-shared attention on B200 (sm_100a).
+ *
+ * The operation (Bat: Efficient Generative Recommender Serving with Bipartite Attention,
+ * lead page, sections "This paper's idea" and "Why it works"): every request holds a user
+ * block and an item block of order-agnostic tokens.  One of the two blocks is the cached
+ * prefix: its K/V is computed once and stored in a cache pool, and every request that
+ * references it computes non-causal softmax attention for its own suffix tokens over
+ *
+ *     out[t, h, :] = softmax_j( scale * q[t, h, :] . [Kp ; Ks][j, h, :] ) [Vp ; Vs][j, h, :]
+ *
+ * where (Kp, Vp) are the rows of its cached prefix and (Ks, Vs) the rows of its own suffix.
+ * There is no mask: the tokens are order-agnostic, which is why either block may serve as
+ * the prefix without changing the result.
+ *
+ * Conventions shared by every entry point
+ *   - Nothing is thrown across the ABI; each call returns a bat_status.  On failure
+ *     bat_last_error() returns a message for the calling thread.
+ *   - Tensors are token-major [T, H, d] with d contiguous (row stride H*d elements).
+ *     They are caller-owned device memory; the library never frees them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
+ *     device work is enqueued on it; no entry point synchronises unless it says so.
+ *   - bf16 tensors: d in {64, 128}; run on tcgen05 tensor cores with fp32 accumulation.
+ *     fp32 tensors: d in {32, 64, 128}; run in fp32 on the CUDA cores (exact fp32 softmax).
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef BAT_H_
+#define BAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BAT_OK = 0,
+  BAT_ERR_INVALID_ARG = 1, /* a pointer, size, table or alignment was rejected */
+  BAT_ERR_UNSUPPORTED = 2, /* valid arguments the library does not implement (e.g. bf16 d=32) */
+  BAT_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+  BAT_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait and returned early */
+  BAT_ERR_OOM = 5          /* a host or device allocation of the library failed */
+} bat_status;
+
+typedef enum { BAT_BF16 = 0, BAT_FP32 = 1 } bat_dtype;
+
+/* Opaque plan: the work list of one batch, produced by the host grouping pass. */
+typedef struct bat_plan bat_plan;
+
+typedef struct {
+  int32_t split_mode;        /* 0 = auto, 1 = never split, 2 = split every splittable item */
+  int32_t split_chunk_tiles; /* 0 = auto; else 128-key tiles per chunk when splitting */
+  int32_t num_sms;           /* 0 = the current device's SM count (148 on B200) */
+  int32_t host_only;         /* 1 = build the work list on the host only (no device upload);
+                                such a plan can be inspected but not run */
+  int32_t reserved[4];       /* must be zero */
+} bat_plan_options;
+
+typedef struct {
+  int64_t n_items;          /* work items (each: one head, up to two 128-row query tiles) */
+  int64_t n_merges;         /* split query tiles whose partials are merged */
+  int64_t n_slots;          /* partial slots in the workspace */
+  int64_t workspace_bytes;  /* bytes bat_attention_forward needs in `workspace` */
+  int64_t total_cost;       /* 128x128 score tiles over all items and heads */
+  int64_t T_suf, T_cache;   /* rows the suffix tensors and the cache must have */
+  int32_t R, P, H, d;
+  int32_t dtype;            /* bat_dtype */
+  int32_t on_device;        /* 1 when the work list was uploaded */
+} bat_plan_info_t;
+
+/*
+ * bat_prefix_kv_build - pack the K/V of `num_prefixes` newly cached prefixes into the pool.
+ * Section "Problem" of the lead page: the K/V of a shared prefix is computed once and
+ * reused.  Prefix i's rows src[src_offsets[i] .. src_offsets[i+1]) of k_src/v_src are
+ * copied to rows dst_offsets[i] .. dst_offsets[i] + len of k_cache/v_cache.
+ *   k_src, v_src      device, [T_src, H, d] of dtype `dt` (read)
+ *   src_offsets       HOST int64 [num_prefixes + 1], non-decreasing, src_offsets[0] >= 0
+ *   dst_offsets       HOST int64 [num_prefixes], dst_offsets[i] >= 0
+ *   k_cache, v_cache  device, [T_cache, H, d] of dtype `dt` (written); the caller sizes them
+ * Destination ranges must not overlap each other or the sources.  Asynchronous on `stream`.
+ * Errors: BAT_ERR_INVALID_ARG (null pointer, bad offsets, misalignment), BAT_ERR_CUDA.
+ */
+bat_status bat_prefix_kv_build(const void* k_src, const void* v_src, const int64_t* src_offsets,
+                               int32_t num_prefixes, const int64_t* dst_offsets, int32_t H,
+                               int32_t d, bat_dtype dt, void* k_cache, void* v_cache,
+                               void* stream);
+
+/*
+ * bat_plan_create - host grouping pass over one batch of requests.
+ * Buckets the requests by the prefix they read, pairs their 128-row query tiles into work
+ * items that stream each prefix's K/V tiles once, orders the items heaviest group first,
+ * optionally splits over-long key streams (partials merged by log-sum-exp), and uploads the
+ * work list to the current device on `stream` (the plan owns that device memory).
+ *   req_prefix      HOST int32 [R]; prefix id in [0, P) or -1 for none
+ *   suffix_offsets  HOST int64 [R+1]; request r owns suffix rows [so[r], so[r+1])
+ *   prefix_offsets  HOST int64 [P+1]; prefix p owns cache rows [po[p], po[p+1])
+ *   H, d, dt        heads, head dim and dtype the forward will run with
+ *   opts            NULL for defaults
+ *   out             receives the plan; release it with bat_plan_destroy
+ * R = 0 and empty suffixes are valid (the forward is then a no-op for those rows).
+ * The host arrays are read during the call only.
+ * Errors: BAT_ERR_INVALID_ARG (non-monotone offsets, prefix id out of range, sizes beyond
+ * int32 rows), BAT_ERR_UNSUPPORTED (dtype/d pair), BAT_ERR_OOM, BAT_ERR_CUDA.
+ */
+bat_status bat_plan_create(const int32_t* req_prefix, const int64_t* suffix_offsets,
+                           const int64_t* prefix_offsets, int32_t R, int32_t P, int32_t H,
+                           int32_t d, bat_dtype dt, const bat_plan_options* opts, void* stream,
+                           bat_plan** out);
+
+/* Releases the plan and its device work list.  Synchronises the device first (cudaFree),
+ * so work already enqueued with the plan completes.  NULL is accepted. */
+bat_status bat_plan_destroy(bat_plan* plan);
+
+/* Copies the plan's summary into *info. */
+bat_status bat_plan_info(const bat_plan* plan, bat_plan_info_t* info);
+
+/* Bytes of device workspace bat_attention_forward needs (0 when no item is split). */
+size_t bat_workspace_bytes(const bat_plan* plan);
+
+/* Copies the host copy of the work list (64-byte records, see the library's internal
+ * layout) into `dst` (host) when dst_bytes >= n_items * 64.  Diagnostics and tests only. */
+bat_status bat_plan_items(const bat_plan* plan, void* dst, size_t dst_bytes);
+/* Same for the merge jobs (32-byte records). */
+bat_status bat_plan_merges(const bat_plan* plan, void* dst, size_t dst_bytes);
+
+/*
+ * bat_attention_forward - the hot path: bipartite prefix-shared attention for every
+ * suffix row of the plan's requests.
+ *   q, k_suf, v_suf   device [T_suf, H, d] of dtype dt: each request's own tokens
+ *   k_cache, v_cache  device [T_cache, H, d] of dtype dt: the prefix pool (may be NULL
+ *                     when T_cache = 0)
+ *   scale             softmax scale; <= 0 selects 1/sqrt(d); must be finite
+ *   out               device [T_suf, H, d] of dtype dt (written; rows of empty requests untouched)
+ *   lse               device fp32 [H, T_suf] or NULL: natural-log log-sum-exp of the
+ *                     scaled scores of each row
+ *   workspace         device scratch of at least bat_workspace_bytes(plan) bytes (NULL if 0)
+ * Every row of the K/V tensors that a 128-row tile window can reach must hold finite values:
+ * the kernel loads whole tiles and weights rows outside a segment by exactly 0.
+ * Asynchronous on `stream`.  Device-side wait timeouts are reported by
+ * bat_get_device_status.
+ * Errors: BAT_ERR_INVALID_ARG (null/misaligned pointer, dtype/d differ from the plan's,
+ * workspace too small, plan not on the device), BAT_ERR_CUDA.
+ */
+bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void* k_suf,
+                                 const void* v_suf, const void* k_cache, const void* v_cache,
+                                 float scale, bat_dtype dt, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reports and clears the device-side status word of the
+ * current device: BAT_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last call,
+ * BAT_ERR_CUDA on a CUDA error, else BAT_OK. */
+bat_status bat_get_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, on every spin-wait inside the kernels (default 2e9).
+ * 0 restores the default.  Diagnostics: a tiny value makes the waits run out on purpose. */
+bat_status bat_set_wait_timeout_ns(uint64_t ns);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* bat_last_error(void);
+
+/* ABI version: (major << 16) | minor. */
+int32_t bat_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BAT_H_ */

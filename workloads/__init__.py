@@ -245,3 +245,34 @@ def device_tensors(table: RequestTable, H: int, d: int, dtype: str, seed: int, d
             flat[s:s + n].copy_(torch.randn(n, generator=g, device=device, dtype=torch.float32))
         out[key] = t
     return out
+
+
+def gather_requests(table: RequestTable, tensors: dict, reqs, out=None):
+    """Compact copy of the rows that requests ``reqs`` read, moved to the host.
+
+    Returns ``(sub_table, host_tensors, rows)``: a table over just those requests and the
+    prefixes they reference, their q/k_suf/v_suf rows and the referenced prefix rows (CPU
+    torch tensors in the original dtype), and the original suffix row index of every row of
+    the compact suffix tensors (so outputs can be gathered the same way).  ``out``, when
+    given, is gathered into ``host_tensors['out']``.  Pure data movement.
+    """
+    import torch
+    reqs = np.asarray(reqs, dtype=np.int64)
+    so, po = table.suffix_offsets, table.prefix_offsets
+    rows = np.concatenate([np.arange(so[r], so[r + 1]) for r in reqs]) if len(reqs) else np.zeros(0, np.int64)
+    used = np.unique(table.req_prefix[reqs][table.req_prefix[reqs] >= 0])
+    remap = {int(p): i for i, p in enumerate(used)}
+    crow = np.concatenate([np.arange(po[p], po[p + 1]) for p in used]) if len(used) else np.zeros(0, np.int64)
+    sub = RequestTable(table.prefix_len[used], np.array([remap.get(int(table.req_prefix[r]), -1) for r in reqs]),
+                       table.suffix_len[reqs], table.kind[reqs])
+
+    def take(t, idx):
+        ii = torch.from_numpy(idx).to(t.device)
+        return t.index_select(0, ii).cpu()
+
+    host = {k: take(tensors[k], rows) for k in ("q", "k_suf", "v_suf")}
+    host["k_cache"] = take(tensors["k_cache"], crow)
+    host["v_cache"] = take(tensors["v_cache"], crow)
+    if out is not None:
+        host["out"] = take(out, rows)
+    return sub, host, rows
