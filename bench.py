@@ -1,0 +1,423 @@
+"""Throughput of bipartite prefix-shared attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixed] [--impl reference]
+
+One step is one pass of the forward over one batch of the named workload (default: the
+mixed bipartite batch, 32768 requests, run as the fewest request-disjoint launches that fit
+in device memory).  Prints one JSON line on rank 0.  Under torchrun each rank serves its own
+batch (weak scaling, rank-seeded inputs, no collective on the data path); the step time is
+the max over ranks of device time measured with CUDA events.
+
+``--impl reference`` times the fp64 CPU oracle instead (the reference arm): on rank 0 only,
+on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, gather_requests, host_tensors, make_table, split_launches  # noqa: E402
+
+METRIC = "bipartite-attention TFLOP/s and requests/s on 1 B200; % of bf16 tensor roofline"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2**20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_flops_bytes(tab, H, d, elt):
+    from prefix_shared_attention_b200.metrics import algorithmic_bytes, algorithmic_flops
+    return (algorithmic_flops(tab.prefix_len, tab.req_prefix, tab.suffix_len, H, d),
+            algorithmic_bytes(tab.prefix_len, tab.req_prefix, tab.suffix_len, H, d, elt))
+
+
+def traffic_per_launch(workload, kernel_src):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this exact
+    kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"bat_attn_tc_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    return rec.get("dram_bytes_per_launch") if rec.get("kernel_sha256_16") == h else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def fits_launches(tab, spec, free_bytes, elt):
+    """Fewest equal request-disjoint launches whose suffix tensors (q, k, v, out) fit next to
+    the resident prefix cache in 80 % of free device memory."""
+    row = spec.H * spec.d * elt
+    cache = 2 * tab.T_cache * row
+    budget = 0.80 * free_bytes - cache - (1 << 30)
+    for n in range(1, 257):
+        if tab.R % n:
+            continue
+        parts = split_launches(tab, n)
+        if 4 * max(p.T_suf for p in parts) * row <= budget:
+            return n
+    raise RuntimeError("workload does not fit in device memory")
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline): the fp64 oracle as it stands, on a bounded sample
+
+def oracle_sample(workload, target_s=12.0, seed=99):
+    """Seeded sample of requests (stratified by prefix kind), its host inputs, and its FLOPs."""
+    import oracle
+    spec = CONFIGS[workload]
+    tab = make_table(workload)
+    rng = np.random.default_rng(seed)
+    order = []
+    kinds = np.unique(tab.kind)
+    per_kind = [rng.permutation(np.flatnonzero(tab.kind == k)) for k in kinds]
+    for i in range(max(len(p) for p in per_kind)):
+        for p in per_kind:
+            if i < len(p):
+                order.append(int(p[i]))
+    order = np.array(order)
+
+    def build(reqs):
+        sub = tab.subset(reqs)
+        used = np.unique(sub.req_prefix[sub.req_prefix >= 0])
+        remap = np.full(tab.P, -1, np.int64)
+        remap[used] = np.arange(len(used))
+        from workloads import RequestTable
+        t = RequestTable(tab.prefix_len[used], np.where(sub.req_prefix >= 0, remap[sub.req_prefix], -1),
+                         sub.suffix_len, sub.kind)
+        x = host_tensors(t, spec.H, spec.d, spec.dtype, spec.seed + 5)
+        x = {k: v.double().numpy() for k, v in x.items()}
+        return t, x
+
+    def run(t, x):
+        return oracle.bipartite_attention(x["q"], x["k_suf"], x["v_suf"], x["k_cache"], x["v_cache"],
+                                          t.prefix_offsets, t.suffix_offsets, t.req_prefix)
+
+    # Calibrate on one request, then take enough requests for about target_s of CPU work.
+    t1, x1 = build(order[:1])
+    f1 = workload_flops_bytes(t1, spec.H, spec.d, 2)[0]
+    s0 = time.perf_counter()
+    run(t1, x1)
+    rate = f1 / max(time.perf_counter() - s0, 1e-6)
+    n = 1
+    flops = f1
+    fl_all = [workload_flops_bytes(tab.subset(order[i:i + 1]), spec.H, spec.d, 2)[0] for i in range(min(len(order), 4096))]
+    while n < len(fl_all) and flops + fl_all[n] <= rate * target_s:
+        flops += fl_all[n]
+        n += 1
+    t, x = build(order[:n])
+    return spec, tab, t, x, run, n
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(workload, target_s=12.0):
+    spec, tab, t, x, run, n = oracle_sample(workload, target_s)
+    flops = workload_flops_bytes(t, spec.H, spec.d, 2)[0]
+    s0 = time.perf_counter()
+    run(t, x)
+    dt = time.perf_counter() - s0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} of {tab.R} requests of '{workload}' (stratified by prefix kind), fp64 numpy, "
+                      f"{flops / 1e9:.1f} GFLOP in {dt:.2f} s",
+            "requests_per_s": n / dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    spec, tab, t, x, run, n = oracle_sample(args.workload, target_s=max(5.0, 150.0 / max(args.steps + args.warmup, 1)))
+    flops = workload_flops_bytes(t, spec.H, spec.d, 2)[0]
+    for _ in range(args.warmup):
+        run(t, x)
+    s0 = time.perf_counter()
+    for _ in range(args.steps):
+        run(t, x)
+    dt = time.perf_counter() - s0
+    value = flops * args.steps / dt / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_requests": n, "requests": tab.R, "H": spec.H, "d": spec.d},
+            "requests_per_s": n * args.steps / dt,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{n} of {tab.R} requests per step, fp64 numpy oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------------
+# GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="mixed", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launches", type=int, default=0, help="override the number of launches per step")
+    args = ap.parse_args()
+    assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("BAT_BENCH_ALLOW_SHORT"), \
+        "at least 3 warm-up steps"
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import prefix_shared_attention_b200 as bat
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    spec = CONFIGS[args.workload]
+    assert spec.dtype == "bf16", "the bench times the bf16 tensor-core path"
+    elt = 2
+    tab = make_table(args.workload)
+    free, total = torch.cuda.mem_get_info()
+    n_launch = args.launches or fits_launches(tab, spec, free, elt)
+    parts = split_launches(tab, n_launch)
+    seed = spec.seed + 1000 * rank
+
+    from workloads import device_tensors
+    cache = device_tensors(tab, spec.H, spec.d, spec.dtype, seed, device=dev, which=("k_cache", "v_cache"))
+    rows = max(p.T_suf for p in parts)
+    suf = device_tensors(parts[0], spec.H, spec.d, spec.dtype, seed + 1, device=dev, which=("q", "k_suf", "v_suf"),
+                         rows=rows)
+    out = torch.empty_like(suf["q"])
+    plans = [bat.Plan(p.req_prefix, p.suffix_offsets, p.prefix_offsets, spec.H, spec.d, bat.BAT_BF16) for p in parts]
+    ws_bytes = max(pl.workspace_bytes for pl in plans)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    launches_per_step = sum(1 + (pl.info().n_merges > 0) for pl in plans)
+    flops_l, bytes_l = zip(*[workload_flops_bytes(p, spec.H, spec.d, elt) for p in parts])
+    step_flops, step_bytes = float(sum(flops_l)), float(sum(bytes_l))
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for i, (p, pl) in enumerate(zip(parts, plans)):
+            T = p.T_suf
+            if events is not None:
+                events[i][0].record(stream)
+            bat.bat_attention_forward(pl, suf["q"][:T], suf["k_suf"][:T], suf["v_suf"][:T], cache["k_cache"],
+                                      cache["v_cache"], out=out[:T], workspace=ws, stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if bat.bat_get_device_status() != bat.BAT_OK:
+        raise RuntimeError(bat.last_error())
+
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in parts] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(ev[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    status = bat.bat_get_device_status()
+    if status != bat.BAT_OK:
+        raise RuntimeError(bat.last_error())
+    elapsed_ms = t0.elapsed_time(t1)
+    kernel_ms = [sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps)) / args.steps
+                 for i in range(len(parts))]
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+
+    ms_per_step = elapsed_ms / args.steps
+    value = step_flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
+    req_s = tab.R * world * args.steps / (elapsed_ms * 1e-3)
+    peaks, peak_kind = load_peaks()
+    achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
+    traffic = traffic_per_launch(args.workload, kernel_src)
+
+    # End to end through the public API with host buffers: per launch, H2D of the request
+    # tokens (q, k, v) from pinned memory, the forward, D2H of the output.  The prefix cache is
+    # resident (it is built once per cached prefix, off this path).
+    e2e = None
+    need_host = 4 * rows * spec.H * spec.d * 2
+    try:
+        import psutil
+        host_ok = psutil.virtual_memory().available > 1.5 * need_host
+    except Exception:
+        host_ok = True
+    if not args.no_e2e and not host_ok:
+        e2e = {"value": None, "unit": UNIT, "skipped": f"needs {need_host / 1e9:.0f} GB of pinned host memory"}
+    elif not args.no_e2e:
+        h = {k: torch.empty((rows, spec.H, spec.d), dtype=torch.bfloat16, pin_memory=True) for k in ("q", "k", "v", "o")}
+        for k, src in (("q", "q"), ("k", "k_suf"), ("v", "v_suf")):
+            h[k].copy_(suf[src])
+
+        def e2e_step():
+            for p, pl in zip(parts, plans):
+                T = p.T_suf
+                suf["q"][:T].copy_(h["q"][:T], non_blocking=True)
+                suf["k_suf"][:T].copy_(h["k"][:T], non_blocking=True)
+                suf["v_suf"][:T].copy_(h["v"][:T], non_blocking=True)
+                bat.bat_attention_forward(pl, suf["q"][:T], suf["k_suf"][:T], suf["v_suf"][:T], cache["k_cache"],
+                                          cache["v_cache"], out=out[:T], workspace=ws, stream=stream)
+                h["o"][:T].copy_(out[:T], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        row_b = spec.H * spec.d * 2
+        e2e = {"value": step_flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(3 * tab.T_suf * row_b), "d2h_bytes_per_step": int(tab.T_suf * row_b),
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+        del h
+        if bat.bat_get_device_status() != bat.BAT_OK:
+            raise RuntimeError(bat.last_error())
+
+    for pl in plans:
+        pl.close()
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del suf, cache, out, ws
+        torch.cuda.empty_cache()
+        base = cpu_baseline(args.workload)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
+                       "prefixes_cached": tab.P, "tokens_suffix": tab.T_suf, "tokens_cache": tab.T_cache,
+                       "l2": "inputs larger than L2 (%.0f GB per launch)" % (step_bytes / n_launch / 1e9),
+                       "parallelism": f"dp{world}" if world > 1 else "single"},
+            "requests_per_s": req_s,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "kernel": "bat_attn_tc_kernel", "kernel_ms_per_launch": kernel_ms,
+                         "alg_gflop_per_launch": [f / 1e9 for f in flops_l],
+                         "alg_gb_per_launch": [b / 1e9 for b in bytes_l]},
+            "cpu_baseline": base, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -10,7 +10,9 @@
 // query tiles consume every shared tile:
 //
 //   warp 8       TMA producer: Q tiles, then K/V tiles in stream order into a ring
-//   warp 9       MMA issuer (one lane): S = Q.K^T (SS) and O += P.V (TS, P read from TMEM)
+//   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V (TS,
+//                P read from TMEM)
+//   warp 11      idle (it completes the third warpgroup for the register split)
 //   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane)
 //   warps 4..7   softmax + epilogue of tile B
 //
@@ -35,7 +37,36 @@ namespace {
 
 __device__ uint32_t g_status_word;
 
+// Compile-time event trace of CTA 0 (off unless built with -DBAT_TRACE): per role, a list of
+// (code, clock64) pairs; code = event | x << 8 | index << 16.
+#ifdef BAT_TRACE
+constexpr int kTraceCap = 8192;
+__device__ unsigned long long* g_trace;   // [5 roles][kTraceCap][2]
+// The buffer pointer is read once per role (a global load per event would itself stall the
+// traced warp by an L2 round trip).
+__device__ __forceinline__ unsigned long long* trace_base(int role) {
+  return (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && g_trace) ? g_trace + (size_t)role * kTraceCap * 2 : nullptr;
+}
+__device__ __forceinline__ void trace(unsigned long long* tp, int& n, uint32_t ev, uint32_t x, uint32_t idx) {
+  if (tp && n < kTraceCap) {
+    const unsigned long long c = clock64();
+    tp[2 * n] = ev | (x << 8) | (idx << 16);
+    tp[2 * n + 1] = c;
+    ++n;
+  }
+}
+#define BAT_TRACE_INIT(role) unsigned long long* trace_p = trace_base(role)
+#define BAT_TRACE_EV(role, n, ev, x, idx) trace(trace_p, n, ev, x, idx)
+#else
+#define BAT_TRACE_INIT(role) ((void)0)
+#define BAT_TRACE_EV(role, n, ev, x, idx) ((void)0)
+#endif
+
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
+#ifndef BAT_FMA_EXP_PAIRS
+#define BAT_FMA_EXP_PAIRS 0
+#endif
+constexpr int kFmaExpPairs = BAT_FMA_EXP_PAIRS;   // of every 8 score columns, pairs exponentiated on the FMA pipe
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 // ------------------------------------------------------------------------------------
@@ -74,6 +105,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Same test, but a thread whose phase is not complete is suspended (up to the hint, in ns)
+// until it completes, instead of returning at once: waiting warps then leave the issue slots
+// of their sub-partition to the warps that have work.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -129,11 +174,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+__device__ __forceinline__ void tmem_ld128f(uint32_t taddr, float (&r)[128]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]), "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15]), "=f"(r[16]), "=f"(r[17]), "=f"(r[18]), "=f"(r[19]), "=f"(r[20]), "=f"(r[21]), "=f"(r[22]), "=f"(r[23]), "=f"(r[24]), "=f"(r[25]), "=f"(r[26]), "=f"(r[27]), "=f"(r[28]), "=f"(r[29]), "=f"(r[30]), "=f"(r[31]), "=f"(r[32]), "=f"(r[33]), "=f"(r[34]), "=f"(r[35]), "=f"(r[36]), "=f"(r[37]), "=f"(r[38]), "=f"(r[39]), "=f"(r[40]), "=f"(r[41]), "=f"(r[42]), "=f"(r[43]), "=f"(r[44]), "=f"(r[45]), "=f"(r[46]), "=f"(r[47]), "=f"(r[48]), "=f"(r[49]), "=f"(r[50]), "=f"(r[51]), "=f"(r[52]), "=f"(r[53]), "=f"(r[54]), "=f"(r[55]), "=f"(r[56]), "=f"(r[57]), "=f"(r[58]), "=f"(r[59]), "=f"(r[60]), "=f"(r[61]), "=f"(r[62]), "=f"(r[63]), "=f"(r[64]), "=f"(r[65]), "=f"(r[66]), "=f"(r[67]), "=f"(r[68]), "=f"(r[69]), "=f"(r[70]), "=f"(r[71]), "=f"(r[72]), "=f"(r[73]), "=f"(r[74]), "=f"(r[75]), "=f"(r[76]), "=f"(r[77]), "=f"(r[78]), "=f"(r[79]), "=f"(r[80]), "=f"(r[81]), "=f"(r[82]), "=f"(r[83]), "=f"(r[84]), "=f"(r[85]), "=f"(r[86]), "=f"(r[87]), "=f"(r[88]), "=f"(r[89]), "=f"(r[90]), "=f"(r[91]), "=f"(r[92]), "=f"(r[93]), "=f"(r[94]), "=f"(r[95]), "=f"(r[96]), "=f"(r[97]), "=f"(r[98]), "=f"(r[99]), "=f"(r[100]), "=f"(r[101]), "=f"(r[102]), "=f"(r[103]), "=f"(r[104]), "=f"(r[105]), "=f"(r[106]), "=f"(r[107]), "=f"(r[108]), "=f"(r[109]), "=f"(r[110]), "=f"(r[111]), "=f"(r[112]), "=f"(r[113]), "=f"(r[114]), "=f"(r[115]), "=f"(r[116]), "=f"(r[117]), "=f"(r[118]), "=f"(r[119]), "=f"(r[120]), "=f"(r[121]), "=f"(r[122]), "=f"(r[123]), "=f"(r[124]), "=f"(r[125]), "=f"(r[126]), "=f"(r[127])
       : "r"(taddr)
       : "memory");
 }
@@ -152,6 +197,62 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (d0, d1) = (a0, a1) * (b, b) + (c, c) on the packed fp32x2 FMA path.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (a0, a1) += (b0, b1) on the packed fp32x2 add path.
+__device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) on the packed fp32x2 FMA path.
+__device__ __forceinline__ void fma2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// 2^x for a pair, on the FMA pipe (offloads the MUFU).  Cody-Waite reduction: j = round(x)
+// by the 1.5 * 2^23 shifter, f = x - j in [-1/2, 1/2], 2^f by a degree-3 polynomial (relative
+// error 7.5e-5, coefficients from csrc/fit_exp2_poly.py), and 2^j added to the exponent
+// field.  x is clamped at -125 so the exponent field cannot underflow (2^-125 is 0 for every
+// use here: the row's largest term is >= 1).
+constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111251e-01f,
+                kExp2C3 = 5.517166480e-02f;
+__device__ __forceinline__ void exp2_fma2(float& x0, float& x1) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0, t1, j0, j1, f0, f1, p0, p1;
+  fma2v(t0, t1, x0, x1, 1.f, 1.f, kShift, kShift);      // round to nearest integer in the low bits
+  fma2v(j0, j1, t0, t1, 1.f, 1.f, -kShift, -kShift);    // j = round(x)
+  fma2v(f0, f1, j0, j1, -1.f, -1.f, x0, x1);            // f = x - j
+  fma2v(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
+  fma2v(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+  fma2v(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+  x0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  x1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -185,7 +286,7 @@ struct Cfg {
   static constexpr int kPanels = D / 64;                 // 64-element (128-byte) column panels
   static constexpr int kPanelBytes = kTileM * 128;       // 128 rows x 128 bytes
   static constexpr int kTileBytes = kPanels * kPanelBytes;
-  static constexpr int kStages = D == 128 ? 4 : 8;        // K/V ring depth
+  static constexpr int kStages = D == 128 ? 5 : 12;       // K/V ring depth (fills 227 KB)
   static constexpr bool kAliasP = D == 128;               // P overwrites S in TMEM
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
@@ -193,7 +294,7 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t p_col(int x) { return kAliasP ? 128u * x : 384u + 64u * x; }
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 1) + 16;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8) + 16;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kStages) * kTileBytes + kBarBytes;
 };
 
@@ -259,8 +360,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   if (!ok) {
     const uint64_t t0 = global_ns();
     while (true) {
-#pragma unroll 1
-      for (int i = 0; i < 16 && !ok; ++i) ok = mbar_test(bar, parity);
+      ok = mbar_test_suspend(bar, parity);
       if (ok) break;
       if (*c.abort_flag) break;
       if (global_ns() - t0 > c.limit_ns) {
@@ -293,7 +393,8 @@ struct Smem {
   uint64_t* s_free;   // [2]
   uint64_t* p_full;   // [2]
   uint64_t* pv_done;  // [2]
-  uint64_t* drain;
+  uint64_t* drain;    // [2]
+  uint64_t* mufu;     // [2][4]: exponential-phase turns, per query tile and sub-partition
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -355,109 +456,127 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
   __syncwarp();
 }
 
+// MMA issuer of query tile X (warp 9 for A, warp 10 for B).  A single issuing thread would
+// serialise both tiles' bookkeeping against a tensor-core queue only about one instruction
+// deep; with one issuer per tile, one tile's waits and commits overlap the other's MMAs.
+// tcgen05.commit tracks only the committing thread's MMAs, so every K/V slot is released by
+// two arrivals, one per issuer: a commit after its MMAs read the slot, or, for a tile this
+// query tile does not read, a plain arrive once the tile has landed.
 template <int D>
-__device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, uint32_t tmem) {
+__device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, uint32_t tmem, int X) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t ring = 0, qcnt[2] = {0, 0}, s_issued[2] = {0, 0}, pv_issued[2] = {0, 0}, p_seen[2] = {0, 0};
+  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
   bool ok = true;
-  const uint32_t q_base = smem_u32(sm.q), kv_base = smem_u32(sm.kv);
+  int tn = 0;
+  (void)tn;
+  BAT_TRACE_INIT(1 + X);
+  // Descriptors are computed once; per instruction only a constant is added to the start
+  // address field (addresses stay below 256 KiB, so the 14-bit field never carries).
+  const uint64_t qdesc = sdesc_sw128(smem_u32(sm.q) + X * C::kTileBytes, 16, 1024);
+  const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.kv), 16, 1024);
+  const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.kv), C::kPanelBytes, 1024);
+  const uint32_t s_t = tmem + C::s_col(X), o_t = tmem + C::o_col(X), p_t = tmem + C::p_col(X);
+
+  auto release_unread = [&](uint32_t r) {
+    ok = wait_bar(sm.kv_full + r % C::kStages, (r / C::kStages) & 1, ctl);
+    if (ok && lane == 0) mbar_arrive(sm.kv_empty + r % C::kStages);
+    __syncwarp();
+  };
+
   for (int64_t it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
     const WorkItem w = p.items[it];
     const Stream st(w);
-    int s_left[2] = {st.count(0), w.n_q == 2 ? st.count(1) : 0};
-    bool first_s[2] = {true, true}, first_pv[2] = {true, true};
     const uint32_t ring0 = ring;
+    ring += 2u * st.n;
+    if (X >= w.n_q) {
+      for (uint32_t r = ring0; ok && r < ring; ++r) release_unread(r);
+      continue;
+    }
+    int s_left = st.count(X);
+    bool first_s = true, first_pv = true;
+    int pend = -1;   // key tile whose PV is still to be issued
 
-    auto do_s = [&](int j) {
-      int mask, row0;
-      bool from_cache;
-      st.tile(w, j, mask, from_cache, row0);
-      const uint32_t rk = ring0 + 2u * j, s = rk % C::kStages;
-      ok = wait_bar(sm.kv_full + s, (rk / C::kStages) & 1, ctl);
-      if (!ok) return;
-      for (int x = 0; x < 2; ++x) {
-        if (!((mask >> x) & 1)) continue;
-        if (first_s[x]) {
-          ok = wait_bar(sm.q_full + x, qcnt[x] & 1, ctl);
-          if (!ok) return;
-          ++qcnt[x];
-          first_s[x] = false;
-        }
-        if (s_issued[x] > 0) {
-          // The S columns are free once the previous P (aliased) was consumed, or once the
-          // softmax finished reading the previous S (separate P columns).
-          if (C::kAliasP) ok = wait_bar(sm.pv_done + x, (pv_issued[x] - 1) & 1, ctl);
-          else ok = wait_bar(sm.s_free + x, (s_issued[x] - 1) & 1, ctl);
-          if (!ok) return;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t qa = q_base + x * C::kTileBytes, kb = kv_base + s * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::s_col(x), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                   C::kIdescS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(sm.s_full + x);
-          if (s_left[x] == 1) tc_commit(sm.q_empty + x);
-        }
-        __syncwarp();
-        --s_left[x];
-        ++s_issued[x];
-      }
-      if (lane == 0) tc_commit(sm.kv_empty + s);
-      __syncwarp();
-    };
-
-    auto do_pv = [&](int j) {
-      int mask, row0;
-      bool from_cache;
-      st.tile(w, j, mask, from_cache, row0);
-      const uint32_t rv = ring0 + 2u * j + 1, s = rv % C::kStages;
+    // PV of key tile jp: O += P . V, P read from TMEM, V (MN-major) from the ring.
+    auto issue_pv = [&](int jp) {
+      BAT_TRACE_EV(1 + X, tn, 3, X, jp);
+      const uint32_t rv = ring0 + 2u * jp + 1, s = rv % C::kStages;
       ok = wait_bar(sm.kv_full + s, (rv / C::kStages) & 1, ctl);
       if (!ok) return;
-      for (int x = 0; x < 2; ++x) {
-        if (!((mask >> x) & 1)) continue;
-        ok = wait_bar(sm.p_full + x, p_seen[x] & 1, ctl);
-        if (!ok) return;
-        ++p_seen[x];
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t vb = kv_base + s * C::kTileBytes;
+      ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
+      if (!ok) return;
+      ++p_seen;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
+        // 16 keys = two 8-row swizzle groups (2 KiB); LBO steps between 64-column panels.
+        mma_ts(o_t, p_t, vd, C::kIdescPV, first_pv ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < kTileN / 16; ++kk) {
-            // V tile is MN-major for this product: 16 keys = two 8-row swizzle groups (2 KiB);
-            // LBO steps between 64-column panels, SBO between 8-row groups.
-            mma_ts(tmem + C::o_col(x), tmem + C::p_col(x) + kk * 8, sdesc_sw128(vb + kk * 2048, C::kPanelBytes, 1024),
-                   C::kIdescPV, (first_pv[x] && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(sm.pv_done + x);
-        }
-        __syncwarp();
-        first_pv[x] = false;
-        ++pv_issued[x];
+        for (int kk = 1; kk < kTileN / 16; ++kk) mma_ts(o_t, p_t + kk * 8, vd + (uint64_t)(kk * 2048 / 16), C::kIdescPV, 1u);
+        tc_commit(sm.pv_done + X);
+        tc_commit(sm.kv_empty + s);
       }
-      if (lane == 0) tc_commit(sm.kv_empty + s);
       __syncwarp();
+      first_pv = false;
+      BAT_TRACE_EV(1 + X, tn, 1, X, jp);
     };
 
-    for (int j = 0; ok && j <= st.n; ++j) {
-      if (C::kAliasP) {
-        if (j >= 1) do_pv(j - 1);
-        if (ok && j < st.n) do_s(j);
-      } else {
-        if (j < st.n) do_s(j);
-        if (ok && j >= 1) do_pv(j - 1);
+    for (int j = 0; ok && j < st.n; ++j) {
+      int mask, row0;
+      bool from_cache;
+      st.tile(w, j, mask, from_cache, row0);
+      const uint32_t rk = ring0 + 2u * j, ks = rk % C::kStages;
+      if (!((mask >> X) & 1)) {
+        release_unread(rk);
+        if (ok) release_unread(rk + 1);
+        continue;
+      }
+      if (pend >= 0) issue_pv(pend);   // before the K wait: a late K tile must not delay it
+      pend = -1;
+      if (!ok) break;
+      BAT_TRACE_EV(1 + X, tn, 4, X, s_issued);
+      ok = wait_bar(sm.kv_full + ks, (rk / C::kStages) & 1, ctl);
+      if (ok && first_s) {
+        ok = wait_bar(sm.q_full + X, qcnt & 1, ctl);
+        ++qcnt;
+        first_s = false;
+      }
+      // Separate P columns (d = 64): S may be overwritten once the softmax has read the
+      // previous S.  Aliased P (d = 128): this S overwrites the columns the PV issued just
+      // before it reads P from; tcgen05.mma instructions issued by one thread execute in
+      // issue order, so that PV has read its A operand before this S writes its accumulator
+      // (the rule NVIDIA's CUTLASS Blackwell attention mainloop relies on as well).
+      if (ok && !C::kAliasP && s_issued > 0) ok = wait_bar(sm.s_free + X, (s_issued - 1) & 1, ctl);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint64_t kd = kdesc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
+          mma_ss(s_t, qdesc + off, kd + off, C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(sm.s_full + X);
+        if (s_left == 1) tc_commit(sm.q_empty + X);
+        tc_commit(sm.kv_empty + ks);
+      }
+      __syncwarp();
+      BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
+      --s_left;
+      ++s_issued;
+      pend = j;
+      if (s_left == 0) {
+        // Exhausted: issue the last PV now, so its V slot is not held while the other query
+        // tile walks the rest of the item.
+        issue_pv(pend);
+        pend = -1;
       }
     }
-    ring = ring0 + 2u * st.n;
   }
   // Wait for every MMA this warp issued before the CTA frees TMEM.
   if (lane == 0) {
-    tc_commit(sm.drain);
-    drain_bar(sm.drain, 0);
+    tc_commit(sm.drain + X);
+    drain_bar(sm.drain + X, 0);
   }
   __syncwarp();
 }
@@ -471,42 +590,53 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
   const uint32_t tP = tmem + C::p_col(X) + lane_off;
   const uint32_t tO = tmem + C::o_col(X) + lane_off;
   const float sl2 = p.scale_log2;
+  // Warp i of tile A and warp i of tile B run on the same sub-partition and share its MUFU:
+  // while both have a tile at the same position they take turns on the exponentials (A first),
+  // so each runs at the MUFU's full rate while the other waits on its MMAs.
+  const int wq = (threadIdx.x >> 5) & 3;
+  uint64_t* const my_turn = sm.mufu + X * 4 + wq;
+  uint64_t* const other_turn = sm.mufu + (1 - X) * 4 + wq;
+  uint32_t turns = 0;
   uint32_t s_seen = 0, pv_base = 0;
   bool ok = true;
+  int tn = 0;
+  (void)tn;
+  BAT_TRACE_INIT(3 + X);
   for (int64_t it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
     const WorkItem w = p.items[it];
     if (X >= w.n_q) continue;
     const Stream st(w);
     const int nX = st.count(X);
+    const int paired = w.n_q == 2 ? min(st.count(0), st.count(1)) : 0;
     float m = -INFINITY, l = 0.f;
     for (int t = 0; t < nX; ++t) {
       const int valid = st.valid(w, X, t);
       ok = wait_bar(sm.s_full + X, s_seen & 1, ctl);
       if (!ok) break;
+      BAT_TRACE_EV(3 + X, tn, 1, X, s_seen);
       ++s_seen;
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld128(tS, sr);
+      float s[128];
+      tmem_ld128f(tS, s);
+      BAT_TRACE_EV(3 + X, tn, 7, X, s_seen);
       if (!C::kAliasP) {
         tc_fence_before();
         mbar_arrive(sm.s_free + X);
       }
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       if (valid < kTileN) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = c < valid ? s[c] : -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      // Row maximum: eight independent 3-input-max chains (short dependency depth).
+      float mx[8];
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int k = 0; k < 8; ++k) {
+        mx[k] = s[16 * k];
+#pragma unroll
+        for (int i = 1; i < 15; i += 2) mx[k] = max3f(mx[k], s[16 * k + i], s[16 * k + i + 1]);
+        mx[k] = fmaxf(mx[k], s[16 * k + 15]);
       }
-      const float tile_m = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float tile_m = fmaxf(max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), mx[6]), mx[7]) * sl2;
       float m_new = m;
       if (t == 0) m_new = tile_m;
       else if (tile_m > m + kRescaleThreshold) m_new = tile_m;
@@ -529,39 +659,60 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
         tmem_st_wait();
       }
       m = m_new;
+      BAT_TRACE_EV(3 + X, tn, 8, X, s_seen);
+      if (t < paired) {
+        ok = wait_bar(my_turn, (turns & 1) ^ (X == 0 ? 1u : 0u), ctl);
+        if (!ok) break;
+        ++turns;
+      }
+      BAT_TRACE_EV(3 + X, tn, 9, X, s_seen);
       const float nm = -m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        s[c] = ex2(fmaf(s[c], sl2, nm));
-        s[c + 1] = ex2(fmaf(s[c + 1], sl2, nm));
-        s[c + 2] = ex2(fmaf(s[c + 2], sl2, nm));
-        s[c + 3] = ex2(fmaf(s[c + 3], sl2, nm));
-        a0 += s[c];
-        a1 += s[c + 1];
-        a2 += s[c + 2];
-        a3 += s[c + 3];
-      }
-      l += (a0 + a1) + (a2 + a3);
       if (!C::kAliasP && t > 0) {
-        // Separate P columns: the previous P must have been consumed.
+        // Separate P columns: the previous P must have been consumed before it is overwritten.
         ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
       }
-      uint32_t pk[32];
+      // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
+      // stored to TMEM (asynchronously) while the next half's exponentials run.  Of every eight
+      // columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the MUFU.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int c = 64 * h; c < 64 * h + 64; c += 8) {
+#pragma unroll
+          for (int k = 0; k < 8; k += 2) ffma2(s[c + k], s[c + k + 1], s[c + k], s[c + k + 1], sl2, nm);
+#pragma unroll
+          for (int k = 0; k < 8 - 2 * kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
+#pragma unroll
+          for (int k = 8 - 2 * kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
+          fadd2(a0, a1, s[c], s[c + 1]);
+          fadd2(a2, a3, s[c + 2], s[c + 3]);
+          fadd2(a0, a1, s[c + 4], s[c + 5]);
+          fadd2(a2, a3, s[c + 6], s[c + 7]);
+        }
+        if (h == 1) {
+          BAT_TRACE_EV(3 + X, tn, 10, X, s_seen);
+          if (t < paired) {
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(other_turn);
+          }
+        }
+        uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]);
         tmem_st32(tP + 32 * h, pk);
       }
+      l += (a0 + a1) + (a2 + a3);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(sm.p_full + X);
+      BAT_TRACE_EV(3 + X, tn, 2, X, s_seen);
     }
     if (!ok) break;
     // Epilogue: O / l, 16-byte stores of this thread's row.
+    BAT_TRACE_EV(3 + X, tn, 5, X, s_seen);
     ok = wait_bar(sm.pv_done + X, (pv_base + nX - 1) & 1, ctl);
     if (!ok) break;
     tc_fence_after();
@@ -626,14 +777,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.p_full = sm.s_free + 2;
   sm.pv_done = sm.p_full + 2;
   sm.drain = sm.pv_done + 2;
-  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.drain + 1);
+  sm.mufu = sm.drain + 2;
+  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.mufu + 8);
   sm.abort_flag = reinterpret_cast<volatile int*>(sm.tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(sm.kv_full + s, 1);
-      mbar_init(sm.kv_empty + s, 1);
+      mbar_init(sm.kv_empty + s, 2);   // one arrival per MMA issuer
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(sm.q_full + x, 1);
@@ -644,6 +796,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
       mbar_init(sm.pv_done + x, 1);
     }
     mbar_init(sm.drain, 1);
+    mbar_init(sm.drain + 1, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(sm.mufu + i, 1);
     *sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -666,9 +820,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   const uint32_t tmem = *sm.tmem_slot;
   const Ctl ctl{sm.abort_flag, p.status, p.wait_ns};
 
-  if (warp == 8) producer_role<D>(p, sm, ctl);
-  else if (warp == 9) mma_role<D>(p, sm, ctl, tmem);
-  else softmax_role<D>(p, sm, ctl, tmem, warp >> 2);
+  // Register split: the control warpgroup (producer, MMA issuer, two idle warps) gives up
+  // registers to the two softmax warpgroups.  384 threads x 168 at launch = 64512 =
+  // 128 x 104 + 256 x 200.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
+    if (warp == 8) producer_role<D>(p, sm, ctl);
+    else if (warp == 9 || warp == 10) mma_role<D>(p, sm, ctl, tmem, warp - 9);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+    softmax_role<D>(p, sm, ctl, tmem, warp >> 2);
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -684,11 +846,9 @@ size_t attn_tc_smem_bytes(int d) { return d == 128 ? Cfg<128>::kSmemBytes : Cfg<
 cudaError_t launch_attn_tc(int d, const TcParams& p, int grid, cudaStream_t s) {
   if (grid <= 0) return cudaSuccess;
   if (d == 128) {
-    static bool attr = false;   // per process; the attribute is per function, not per device
     cudaError_t e = cudaFuncSetAttribute(bat_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg<128>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    (void)attr;
     bat_attn_tc_kernel<128><<<grid, kTcThreads, Cfg<128>::kSmemBytes, s>>>(p);
   } else if (d == 64) {
     cudaError_t e = cudaFuncSetAttribute(bat_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -700,6 +860,12 @@ cudaError_t launch_attn_tc(int d, const TcParams& p, int grid, cudaStream_t s) {
   }
   return cudaGetLastError();
 }
+
+#ifdef BAT_TRACE
+extern "C" int bat_debug_set_trace(void* buf) {
+  return (int)cudaMemcpyToSymbol(g_trace, &buf, sizeof(buf));
+}
+#endif
 
 cudaError_t device_status_word(uint32_t** out) {
   return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_status_word);

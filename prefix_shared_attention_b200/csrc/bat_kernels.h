@@ -59,7 +59,7 @@ struct PackBatch {
 // Each launcher returns the cudaError_t of the launch.
 cudaError_t launch_attn_tc(int d, const TcParams& p, int grid, cudaStream_t s);
 size_t attn_tc_smem_bytes(int d);
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 384;   // 3 warpgroups: softmax A, softmax B, control
 cudaError_t launch_attn_simt(int d, const SimtParams& p, cudaStream_t s);
 cudaError_t launch_merge(int d, bool out_bf16, const MergeParams& p, cudaStream_t s);
 cudaError_t launch_pack(const void* ks, const void* vs, void* kc, void* vc, const PackBatch& b,
