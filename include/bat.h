@@ -147,6 +147,28 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
                                  float scale, bat_dtype dt, void* out, float* lse,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * bat_attention_forward_noalloc - bat_attention_forward for callers that cannot allocate
+ * device memory (the paper has no counterpart; this is a deployment aid).  Examples: a process
+ * whose device memory is owned by another allocator that reserved the pool, or a serving loop
+ * that must avoid cudaMalloc/cudaFree because they can synchronize the device.  Plans are still
+ * created beforehand with bat_plan_create; this call itself allocates nothing.
+ * Arguments are those of bat_attention_forward without the workspace: the split-path scratch
+ * lives in a fixed 32 MiB array inside the library, held by every GPU that loads it until exit.
+ *   - A plan whose bat_workspace_bytes exceeds 32 MiB is rejected: BAT_ERR_INVALID_ARG, with a
+ *     message in bat_last_error() giving both sizes.
+ *   - All calls on a device share that array; calls whose kernels overlap on the GPU race on
+ *     it, so issue them on one stream.  It keeps the previous call's contents; nothing in it
+ *     needs to start at zero.
+ *   - The first call on each device resolves the array's address (with that device current);
+ *     make it before any stream capture starts on that device.
+ * Errors: those of bat_attention_forward, plus BAT_ERR_CUDA if the address lookup fails.
+ */
+bat_status bat_attention_forward_noalloc(const bat_plan* plan, const void* q, const void* k_suf,
+                                         const void* v_suf, const void* k_cache, const void* v_cache,
+                                         float scale, bat_dtype dt, void* out, float* lse,
+                                         void* stream);
+
 /* Synchronises `stream`, then reports and clears the device-side status word of the
  * current device: BAT_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last call,
  * BAT_ERR_CUDA on a CUDA error, else BAT_OK. */

@@ -22,6 +22,7 @@ from ._bat import (  # noqa: F401
     BatError,
     Plan,
     bat_attention_forward,
+    bat_attention_forward_noalloc,
     bat_get_device_status,
     bat_prefix_kv_build,
     bat_set_wait_timeout_ns,

@@ -59,6 +59,7 @@ _SIGNATURES = {
     "bat_plan_items": (_i32, [_vp, _vp, _sz]),
     "bat_plan_merges": (_i32, [_vp, _vp, _sz]),
     "bat_attention_forward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "bat_attention_forward_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _f32, _i32, _vp, _vp, _vp]),
     "bat_get_device_status": (_i32, [_vp]),
     "bat_set_wait_timeout_ns": (_i32, [_u64]),
     "bat_last_error": (C.c_char_p, []),
@@ -202,6 +203,21 @@ def bat_attention_forward(plan: Plan, q, k_suf, v_suf, k_cache=None, v_cache=Non
                                     float(scale), dtype_code(q.dtype), ptr(out), ptr(lse), ptr(workspace),
                                     int(workspace.numel()) if workspace is not None else 0,
                                     _stream_handle(stream)))
+    return out
+
+
+def bat_attention_forward_noalloc(plan: Plan, q, k_suf, v_suf, k_cache=None, v_cache=None, out=None, lse=None,
+                                  scale: float = 0.0, stream=None):
+    """The forward without a workspace argument: split scratch comes from a fixed array inside
+    the library (for callers that cannot allocate device memory).  ``out`` must be given by
+    callers that cannot allocate; when omitted it is allocated here for convenience."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    check(lib.bat_attention_forward_noalloc(plan.handle, ptr(q), ptr(k_suf), ptr(v_suf), ptr(k_cache), ptr(v_cache),
+                                            float(scale), dtype_code(q.dtype), ptr(out), ptr(lse),
+                                            _stream_handle(stream)))
     return out
 
 

@@ -90,6 +90,11 @@ bat_status encode_map(CUtensorMap* m, const void* base, int64_t T, int32_t H, in
 
 }  // namespace
 
+namespace bat {
+// Sets this thread's bat_last_error() message (for entry points defined in other files).
+void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+}  // namespace bat
+
 extern "C" {
 
 const char* bat_last_error(void) { return g_err.c_str(); }
