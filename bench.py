@@ -242,6 +242,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--launches", type=int, default=0, help="override the number of launches per step")
+    ap.add_argument("--subset", type=int, default=0,
+                    help="profiling aid: only the first N requests (and the prefixes they read); not a bench line")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("BAT_BENCH_ALLOW_SHORT"), \
         "at least 3 warm-up steps"
@@ -266,6 +268,8 @@ def main():
     assert spec.dtype == "bf16", "the bench times the bf16 tensor-core path"
     elt = 2
     tab = make_table(args.workload)
+    if args.subset:
+        tab = tab.compact(np.arange(min(args.subset, tab.R)))
     free, total = torch.cuda.mem_get_info()
     n_launch = args.launches or fits_launches(tab, spec, free, elt)
     parts = split_launches(tab, n_launch)
@@ -399,7 +403,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
+            "config": {"workload": args.workload + (f"[:{args.subset}]" if args.subset else ""), "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
                        "prefixes_cached": tab.P, "tokens_suffix": tab.T_suf, "tokens_cache": tab.T_cache,
                        "l2": "inputs larger than L2 (%.0f GB per launch)" % (step_bytes / n_launch / 1e9),
                        "parallelism": f"dp{world}" if world > 1 else "single"},

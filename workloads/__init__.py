@@ -126,6 +126,16 @@ class RequestTable:
         out[m] = self.prefix_len[self.req_prefix[m]]
         return out
 
+    def compact(self, idx: np.ndarray) -> "RequestTable":
+        """Requests ``idx`` over a cache holding only the prefixes they reference (ids remapped)."""
+        idx = np.asarray(idx, dtype=np.int64)
+        rp = self.req_prefix[idx]
+        used = np.unique(rp[rp >= 0])
+        remap = np.full(max(self.P, 1), -1, np.int64)
+        remap[used] = np.arange(len(used))
+        return RequestTable(self.prefix_len[used], np.where(rp >= 0, remap[np.clip(rp, 0, None)], -1),
+                            self.suffix_len[idx], self.kind[idx], dict(self.note))
+
     def subset(self, idx: np.ndarray) -> "RequestTable":
         """Requests ``idx`` (in that order) over the same prefix cache."""
         idx = np.asarray(idx, dtype=np.int64)
