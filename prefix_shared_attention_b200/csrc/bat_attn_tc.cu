@@ -163,6 +163,40 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// Warp-uniform issue: every lane executes these with identical operands (so they stay in
+// uniform registers) and elect.sync picks the one lane that issues.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b64 st;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
 // 32 consecutive fp32 columns of this thread's TMEM lane, waited for in the same statement
 // so no use of the registers can be scheduled before the data has arrived.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -294,7 +328,7 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t p_col(int x) { return kAliasP ? 128u * x : 384u + 64u * x; }
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8) + 16;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8 + 2) + 16;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kStages) * kTileBytes + kBarBytes;
 };
 
@@ -395,6 +429,7 @@ struct Smem {
   uint64_t* pv_done;  // [2]
   uint64_t* drain;    // [2]
   uint64_t* mufu;     // [2][4]: exponential-phase turns, per query tile and sub-partition
+  uint64_t* iturn;    // [2]: MMA-batch issue turns, per query tile
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -466,7 +501,7 @@ template <int D>
 __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, uint32_t tmem, int X) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
+  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0, iturns = 0;
   bool ok = true;
   int tn = 0;
   (void)tn;
@@ -494,31 +529,33 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       continue;
     }
     int s_left = st.count(X);
+    // While both query tiles have a key tile at the same position, their MMA batches
+    // [PV of the previous tile, S of this tile] alternate A, B through an issue token, so the
+    // S that unblocks one tile's next softmax is not interleaved with the other tile's PV.
+    const int paired = w.n_q == 2 ? min(st.count(0), st.count(1)) : 0;
+    int t = 0;
     bool first_s = true, first_pv = true;
     int pend = -1;   // key tile whose PV is still to be issued
 
-    // PV of key tile jp: O += P . V, P read from TMEM, V (MN-major) from the ring.
-    auto issue_pv = [&](int jp) {
+    // Waits for the PV of key tile jp: its V tile landed and its P is in TMEM.
+    auto wait_pv = [&](int jp) {
       BAT_TRACE_EV(1 + X, tn, 3, X, jp);
-      const uint32_t rv = ring0 + 2u * jp + 1, s = rv % C::kStages;
-      ok = wait_bar(sm.kv_full + s, (rv / C::kStages) & 1, ctl);
-      if (!ok) return;
-      ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
-      if (!ok) return;
+      const uint32_t rv = ring0 + 2u * jp + 1;
+      ok = wait_bar(sm.kv_full + rv % C::kStages, (rv / C::kStages) & 1, ctl);
+      if (ok) ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
       ++p_seen;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
-        // 16 keys = two 8-row swizzle groups (2 KiB); LBO steps between 64-column panels.
-        mma_ts(o_t, p_t, vd, C::kIdescPV, first_pv ? 0u : 1u);
+    };
+    // PV of key tile jp (lane 0): O += P . V, P read from TMEM, V (MN-major) from the ring.
+    auto emit_pv = [&](int jp) {
+      const uint32_t s = (ring0 + 2u * jp + 1) % C::kStages;
+      const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
+      // 16 keys = two 8-row swizzle groups (2 KiB); LBO steps between 64-column panels.
+      mma_ts_w(o_t, p_t, vd, C::kIdescPV, first_pv ? 0u : 1u);
 #pragma unroll
-        for (int kk = 1; kk < kTileN / 16; ++kk) mma_ts(o_t, p_t + kk * 8, vd + (uint64_t)(kk * 2048 / 16), C::kIdescPV, 1u);
-        tc_commit(sm.pv_done + X);
-        tc_commit(sm.kv_empty + s);
-      }
-      __syncwarp();
-      first_pv = false;
-      BAT_TRACE_EV(1 + X, tn, 1, X, jp);
+      for (int kk = 1; kk < kTileN / 16; ++kk)
+        mma_ts_w(o_t, p_t + kk * 8, vd + (uint64_t)(kk * 2048 / 16), C::kIdescPV, 1u);
+      tc_commit_w(sm.pv_done + X);
+      tc_commit_w(sm.kv_empty + s);
     };
 
     for (int j = 0; ok && j < st.n; ++j) {
@@ -531,11 +568,9 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         if (ok) release_unread(rk + 1);
         continue;
       }
-      if (pend >= 0) issue_pv(pend);   // before the K wait: a late K tile must not delay it
-      pend = -1;
-      if (!ok) break;
+      if (pend >= 0) wait_pv(pend);
       BAT_TRACE_EV(1 + X, tn, 4, X, s_issued);
-      ok = wait_bar(sm.kv_full + ks, (rk / C::kStages) & 1, ctl);
+      if (ok) ok = wait_bar(sm.kv_full + ks, (rk / C::kStages) & 1, ctl);
       if (ok && first_s) {
         ok = wait_bar(sm.q_full + X, qcnt & 1, ctl);
         ++qcnt;
@@ -547,28 +582,42 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       // issue order, so that PV has read its A operand before this S writes its accumulator
       // (the rule NVIDIA's CUTLASS Blackwell attention mainloop relies on as well).
       if (ok && !C::kAliasP && s_issued > 0) ok = wait_bar(sm.s_free + X, (s_issued - 1) & 1, ctl);
+      if (ok && t < paired) {
+        ok = wait_bar(sm.iturn + X, (iturns & 1) ^ (X == 0 ? 1u : 0u), ctl);
+        ++iturns;
+      }
       if (!ok) break;
       tc_fence_after();
-      if (lane == 0) {
+      if (pend >= 0) emit_pv(pend);
+      {
         const uint64_t kd = kdesc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
-          mma_ss(s_t, qdesc + off, kd + off, C::kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss_w(s_t, qdesc + off, kd + off, C::kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(sm.s_full + X);
-        if (s_left == 1) tc_commit(sm.q_empty + X);
-        tc_commit(sm.kv_empty + ks);
+        tc_commit_w(sm.s_full + X);
+        if (s_left == 1) tc_commit_w(sm.q_empty + X);
+        tc_commit_w(sm.kv_empty + ks);
+        if (t < paired) mbar_arrive_w(sm.iturn + (1 - X));
       }
       __syncwarp();
+      if (pend >= 0) first_pv = false;
       BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
       --s_left;
       ++s_issued;
+      ++t;
       pend = j;
       if (s_left == 0) {
         // Exhausted: issue the last PV now, so its V slot is not held while the other query
         // tile walks the rest of the item.
-        issue_pv(pend);
+        wait_pv(pend);
+        if (!ok) break;
+        tc_fence_after();
+        emit_pv(pend);
+        __syncwarp();
+        first_pv = false;
+        BAT_TRACE_EV(1 + X, tn, 1, X, pend);
         pend = -1;
       }
     }
@@ -778,7 +827,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.pv_done = sm.p_full + 2;
   sm.drain = sm.pv_done + 2;
   sm.mufu = sm.drain + 2;
-  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.mufu + 8);
+  sm.iturn = sm.mufu + 8;
+  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.iturn + 2);
   sm.abort_flag = reinterpret_cast<volatile int*>(sm.tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -798,6 +848,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     mbar_init(sm.drain, 1);
     mbar_init(sm.drain + 1, 1);
     for (int i = 0; i < 8; ++i) mbar_init(sm.mufu + i, 1);
+    mbar_init(sm.iturn, 1);
+    mbar_init(sm.iturn + 1, 1);
     *sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
