@@ -67,6 +67,14 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 betwee
 #define BAT_FMA_EXP_PAIRS 0
 #endif
 constexpr int kFmaExpPairs = BAT_FMA_EXP_PAIRS;   // of every 8 score columns, pairs exponentiated on the FMA pipe
+#ifndef BAT_MUFU_TURNS
+#define BAT_MUFU_TURNS 0
+#endif
+#ifndef BAT_ISSUE_TOKEN
+#define BAT_ISSUE_TOKEN 1
+#endif
+constexpr bool kMufuTurns = BAT_MUFU_TURNS != 0;   // the two query tiles alternate on the MUFU
+constexpr bool kIssueToken = BAT_ISSUE_TOKEN != 0; // the two MMA issuers alternate [PV, S] batches
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 // ------------------------------------------------------------------------------------
@@ -532,7 +540,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
     // While both query tiles have a key tile at the same position, their MMA batches
     // [PV of the previous tile, S of this tile] alternate A, B through an issue token, so the
     // S that unblocks one tile's next softmax is not interleaved with the other tile's PV.
-    const int paired = w.n_q == 2 ? min(st.count(0), st.count(1)) : 0;
+    const int paired = (kIssueToken && w.n_q == 2) ? min(st.count(0), st.count(1)) : 0;
     int t = 0;
     bool first_s = true, first_pv = true;
     int pend = -1;   // key tile whose PV is still to be issued
@@ -656,7 +664,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     if (X >= w.n_q) continue;
     const Stream st(w);
     const int nX = st.count(X);
-    const int paired = w.n_q == 2 ? min(st.count(0), st.count(1)) : 0;
+    const int paired = (kMufuTurns && w.n_q == 2) ? min(st.count(0), st.count(1)) : 0;
     float m = -INFINITY, l = 0.f;
     for (int t = 0; t < nX; ++t) {
       const int valid = st.valid(w, X, t);
