@@ -22,6 +22,7 @@ struct bat_plan {
   bat::PlanResult host;
   bat::WorkItem* d_items = nullptr;
   bat::MergeJob* d_merges = nullptr;
+  int32_t* d_counter = nullptr;   // work-item counter of the attention kernel
   int32_t R = 0, P = 0, H = 0, d = 0;
   bat_dtype dt = BAT_BF16;
   int64_t T_suf = 0, T_cache = 0;
@@ -211,11 +212,13 @@ bat_status bat_plan_create(const int32_t* req_prefix, const int64_t* suffix_offs
     const size_t ib = plan->host.n_items * sizeof(bat::WorkItem), mb = plan->host.n_merges * sizeof(bat::MergeJob);
     if (ib) e = cudaMalloc(&plan->d_items, ib);
     if (e == cudaSuccess && mb) e = cudaMalloc(&plan->d_merges, mb);
+    if (e == cudaSuccess) e = cudaMalloc(&plan->d_counter, 16);
     if (e == cudaSuccess && ib) e = cudaMemcpyAsync(plan->d_items, plan->host.items, ib, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && mb) e = cudaMemcpyAsync(plan->d_merges, plan->host.merges, mb, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) {
       cudaFree(plan->d_items);
       cudaFree(plan->d_merges);
+      cudaFree(plan->d_counter);
       bat::free_plan_result(&plan->host);
       delete plan;
       return e == cudaErrorMemoryAllocation ? fail(BAT_ERR_OOM, "device allocation of the work list failed")
@@ -236,6 +239,7 @@ bat_status bat_plan_destroy(bat_plan* plan) {
     cudaGetDevice(&cur);
     if (cur != plan->device) cudaSetDevice(plan->device);
     cudaError_t e1 = cudaFree(plan->d_items), e2 = cudaFree(plan->d_merges);
+    cudaFree(plan->d_counter);
     if (cur >= 0 && cur != plan->device) cudaSetDevice(cur);
     if (e1 != cudaSuccess || e2 != cudaSuccess) st = cuda_fail(e1 != cudaSuccess ? e1 : e2, "cudaFree of the work list");
   }
@@ -345,6 +349,9 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
     p.scale_log2 = sc * 1.4426950408889634f;
     p.status = status;
     p.wait_ns = g_wait_ns.load();
+    p.item_counter = plan->d_counter;
+    e = cudaMemsetAsync(plan->d_counter, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "resetting the work-item counter");
     const int grid = (int)std::min<int64_t>(plan->host.n_items, plan->num_sms);
     e = bat::launch_attn_tc(plan->d, p, grid, s);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");

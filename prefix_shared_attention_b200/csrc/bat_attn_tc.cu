@@ -63,6 +63,8 @@ __device__ __forceinline__ void trace(unsigned long long* tp, int& n, uint32_t e
 #endif
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
+constexpr int kItemQ = 4;                   // work items the producer may run ahead by
+constexpr int kItemConsumers = 10;          // 2 MMA warps + 8 softmax warps pop every item
 #ifndef BAT_FMA_EXP_PAIRS
 #define BAT_FMA_EXP_PAIRS 0
 #endif
@@ -336,7 +338,7 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t p_col(int x) { return kAliasP ? 128u * x : 384u + 64u * x; }
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8 + 2) + 16;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kStages) * kTileBytes + kBarBytes;
 };
 
@@ -438,9 +440,27 @@ struct Smem {
   uint64_t* drain;    // [2]
   uint64_t* mufu;     // [2][4]: exponential-phase turns, per query tile and sub-partition
   uint64_t* iturn;    // [2]: MMA-batch issue turns, per query tile
+  uint64_t* itq_full;   // [kItemQ]
+  uint64_t* itq_empty;  // [kItemQ]
+  volatile int* itq;    // [kItemQ] work-item indices handed from the producer to the others
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
+
+// Work items are handed out dynamically (a global counter), so items next to each other in
+// the list (same prefix group, same head) run at the same time on different CTAs and share
+// their prefix and suffix tiles through L2.  The producer warp takes the next index and
+// passes it to the MMA and softmax warps through a small queue; -1 ends the kernel.
+template <int D>
+__device__ __forceinline__ int pop_item(const Smem<D>& sm, uint32_t& k, const Ctl& ctl, bool& ok) {
+  const uint32_t slot = k % kItemQ;
+  ok = wait_bar(sm.itq_full + slot, (k / kItemQ) & 1, ctl);
+  const int it = ok ? sm.itq[slot] : -1;
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(sm.itq_empty + slot);
+  ++k;
+  return it;
+}
 
 // ------------------------------------------------------------------------------------
 // Roles
@@ -449,9 +469,23 @@ template <int D>
 __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t ring = 0, qcnt[2] = {0, 0};
+  uint32_t ring = 0, qcnt[2] = {0, 0}, kq = 0;
   bool ok = true;
-  for (int64_t it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+  while (ok) {
+    const uint32_t slot = kq % kItemQ;
+    ok = wait_bar(sm.itq_empty + slot, ((kq / kItemQ) & 1) ^ 1, ctl);
+    if (!ok) break;
+    int it = 0;
+    if (lane == 0) it = atomicAdd(p.item_counter, 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    const bool done = it >= p.n_items;
+    if (lane == 0) {
+      sm.itq[slot] = done ? -1 : it;
+      mbar_arrive(sm.itq_full + slot);
+    }
+    __syncwarp();
+    ++kq;
+    if (done) break;
     const WorkItem w = p.items[it];
     for (int x = 0; ok && x < w.n_q; ++x) {
       ok = wait_bar(sm.q_empty + x, (qcnt[x] & 1) ^ 1, ctl);
@@ -527,7 +561,10 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
     __syncwarp();
   };
 
-  for (int64_t it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+  uint32_t kq = 0;
+  while (ok) {
+    const int it = pop_item<D>(sm, kq, ctl, ok);
+    if (it < 0) break;
     const WorkItem w = p.items[it];
     const Stream st(w);
     const uint32_t ring0 = ring;
@@ -659,7 +696,10 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
   int tn = 0;
   (void)tn;
   BAT_TRACE_INIT(3 + X);
-  for (int64_t it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+  uint32_t kq = 0;
+  while (ok) {
+    const int it = pop_item<D>(sm, kq, ctl, ok);
+    if (it < 0) break;
     const WorkItem w = p.items[it];
     if (X >= w.n_q) continue;
     const Stream st(w);
@@ -836,7 +876,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.drain = sm.pv_done + 2;
   sm.mufu = sm.drain + 2;
   sm.iturn = sm.mufu + 8;
-  sm.tmem_slot = reinterpret_cast<uint32_t*>(sm.iturn + 2);
+  sm.itq_full = sm.iturn + 2;
+  sm.itq_empty = sm.itq_full + kItemQ;
+  sm.itq = reinterpret_cast<volatile int*>(sm.itq_empty + kItemQ);
+  sm.tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(sm.itq) + kItemQ);
   sm.abort_flag = reinterpret_cast<volatile int*>(sm.tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -858,6 +901,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     for (int i = 0; i < 8; ++i) mbar_init(sm.mufu + i, 1);
     mbar_init(sm.iturn, 1);
     mbar_init(sm.iturn + 1, 1);
+    for (int i = 0; i < kItemQ; ++i) {
+      mbar_init(sm.itq_full + i, 1);
+      mbar_init(sm.itq_empty + i, kItemConsumers);
+    }
     *sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }

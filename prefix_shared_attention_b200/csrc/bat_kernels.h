@@ -22,6 +22,7 @@ struct alignas(64) TcParams {
   int32_t pad0;
   uint32_t* status;     // device status word (bit 0: a wait timed out)
   uint64_t wait_ns;     // bound on every spin-wait
+  int32_t* item_counter;  // next work item to hand out (zeroed before each launch)
 };
 
 // CUDA-core fp32 path, d in {32, 64, 128}.
