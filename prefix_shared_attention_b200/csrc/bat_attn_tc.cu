@@ -613,7 +613,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         if (ok) release_unread(rk + 1);
         continue;
       }
-      if (pend >= 0) wait_pv(pend);
+      if (C::kAliasP && pend >= 0) wait_pv(pend);
       BAT_TRACE_EV(1 + X, tn, 4, X, s_issued);
       if (ok) ok = wait_bar(sm.kv_full + ks, (rk / C::kStages) & 1, ctl);
       if (ok && first_s) {
@@ -633,7 +633,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       }
       if (!ok) break;
       tc_fence_after();
-      if (pend >= 0) emit_pv(pend);
+      if (C::kAliasP && pend >= 0) emit_pv(pend);
       {
         const uint64_t kd = kdesc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
 #pragma unroll
@@ -647,6 +647,16 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         if (t < paired) mbar_arrive_w(sm.iturn + (1 - X));
       }
       __syncwarp();
+      if (!C::kAliasP && pend >= 0) {
+        // Separate P columns: S of this tile went first (the softmax had read the previous S),
+        // so it is computed while the softmax still works on the previous tile; the previous
+        // tile's PV follows as soon as its P is written.
+        wait_pv(pend);
+        if (!ok) break;
+        tc_fence_after();
+        emit_pv(pend);
+        __syncwarp();
+      }
       if (pend >= 0) first_pv = false;
       BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
       --s_left;
@@ -765,12 +775,6 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       BAT_TRACE_EV(3 + X, tn, 9, X, s_seen);
       const float nm = -m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      if (!C::kAliasP && t > 0) {
-        // Separate P columns: the previous P must have been consumed before it is overwritten.
-        ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
-        if (!ok) break;
-        tc_fence_after();
-      }
       // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
       // stored to TMEM (asynchronously) while the next half's exponentials run.  Of every eight
       // columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the MUFU.
@@ -796,11 +800,18 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
             if ((threadIdx.x & 31) == 0) mbar_arrive(other_turn);
           }
         }
+        if (!C::kAliasP && t > 0 && h == 0) {
+          // Separate P columns: the previous P must have been consumed before it is overwritten.
+          ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+        }
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]);
         tmem_st32(tP + 32 * h, pk);
       }
+      if (!ok) break;
       l += (a0 + a1) + (a2 + a3);
       tmem_st_wait();
       tc_fence_before();
