@@ -9,15 +9,20 @@
 // The CTA streams the item's key tiles through shared memory with TMA, once each, and both
 // query tiles consume every shared tile:
 //
-//   warp 8       TMA producer: Q tiles, then K/V tiles in stream order into a ring
-//   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V (TS,
-//                P read from TMEM)
+//   warp 8       TMA producer: Q tiles, then K/V tiles into a ring in the order the MMA
+//                issuers consume them: K0, K1, V0, K2, V1, ... (the K tile of key tile j+1
+//                ahead of the V tile of key tile j)
+//   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V
+//                (d = 128: SS, P read from shared memory; d = 64: TS, P read from TMEM).  S of
+//                key tile j+1 is issued as soon as the softmax has read S of tile j, so it is
+//                computed while the softmax of tile j runs; PV of tile j follows its P.
 //   warp 11      idle (it completes the third warpgroup for the register split)
 //   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane)
 //   warps 4..7   softmax + epilogue of tile B
 //
-// TMEM (512 columns): S_A, S_B (128 fp32 columns each), O_A, O_B (d columns each); P (bf16
-// pairs, 64 columns) aliases S when d = 128, and has its own columns when d = 64.
+// TMEM (512 columns): S_A, S_B (128 fp32 columns each), O_A, O_B (d columns each); at d = 64
+// P (bf16 pairs, 64 columns per tile) takes the remaining 128 columns, at d = 128 P lives in
+// shared memory (one 32 KiB tile per query tile) because TMEM is full.
 // The softmax is online in the base-2 domain with a lazily updated reference maximum: the
 // accumulator is rescaled only when a row's maximum grows by more than kRescaleThreshold,
 // which is exact because O and the row sum l always share the same reference.
@@ -65,18 +70,11 @@ __device__ __forceinline__ void trace(unsigned long long* tp, int& n, uint32_t e
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
 constexpr int kItemQ = 4;                   // work items the producer may run ahead by
 constexpr int kItemConsumers = 10;          // 2 MMA warps + 8 softmax warps pop every item
-#ifndef BAT_FMA_EXP_PAIRS
-#define BAT_FMA_EXP_PAIRS 0
+#ifdef BAT_FMA_EXP_PAIRS
+constexpr int kFmaExpPairsSet = BAT_FMA_EXP_PAIRS;   // build-time override, same for every d
+#else
+constexpr int kFmaExpPairsSet = -1;
 #endif
-constexpr int kFmaExpPairs = BAT_FMA_EXP_PAIRS;   // of every 8 score columns, pairs exponentiated on the FMA pipe
-#ifndef BAT_MUFU_TURNS
-#define BAT_MUFU_TURNS 0
-#endif
-#ifndef BAT_ISSUE_TOKEN
-#define BAT_ISSUE_TOKEN 1
-#endif
-constexpr bool kMufuTurns = BAT_MUFU_TURNS != 0;   // the two query tiles alternate on the MUFU
-constexpr bool kIssueToken = BAT_ISSUE_TOKEN != 0; // the two MMA issuers alternate [PV, S] batches
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 // ------------------------------------------------------------------------------------
@@ -227,6 +225,10 @@ __device__ __forceinline__ void tmem_ld128f(uint32_t taddr, float (&r)[128]) {
       : "memory");
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
@@ -330,16 +332,21 @@ struct Cfg {
   static constexpr int kPanels = D / 64;                 // 64-element (128-byte) column panels
   static constexpr int kPanelBytes = kTileM * 128;       // 128 rows x 128 bytes
   static constexpr int kTileBytes = kPanels * kPanelBytes;
-  static constexpr int kStages = D == 128 ? 5 : 12;       // K/V ring depth (fills 227 KB)
-  static constexpr bool kAliasP = D == 128;               // P overwrites S in TMEM
+  static constexpr bool kPSmem = D == 128;                // P in shared memory (TMEM is full)
+  static constexpr int kPBufs = kPSmem ? 2 : 0;            // P tiles in shared memory
+  static constexpr int kStages = D == 128 ? 3 : 12;        // K/V ring depth (fills 227 KB)
+  // Of every 8 score columns, pairs exponentiated on the FMA pipe (the rest on the MUFU): at
+  // d = 64 the MUFU is the busier unit (its exponentials take twice the MMA time).
+  static constexpr int kFmaExpPairs = kFmaExpPairsSet >= 0 ? kFmaExpPairsSet : (D == 64 ? 1 : 0);
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
   __host__ __device__ static constexpr uint32_t o_col(int x) { return 256u + (uint32_t)D * x; }
-  __host__ __device__ static constexpr uint32_t p_col(int x) { return kAliasP ? 128u * x : 384u + 64u * x; }
+  __host__ __device__ static constexpr uint32_t p_col(int x) { return 384u + 64u * x; }   // d = 64 only
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 8 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
-  static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kStages) * kTileBytes + kBarBytes;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kPBufs + kStages) * kTileBytes + kBarBytes;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 // The key tiles an item streams: prefix tiles (read by every query tile of the item), then
@@ -382,6 +389,24 @@ struct Stream {
     }
     mask = 1 << x;
     row0 = (x ? w.sB_row0 : w.sA_row0) + idx * kTileN;
+  }
+  // Ring position pos (0 .. 2n-1) of the item's K/V loads: K0, K1, V0, K2, V1, ..., K(n-1),
+  // V(n-2), V(n-1).  This is the order in which each MMA issuer uses them (S of key tile j+1,
+  // then PV of key tile j), so every issuer walks the ring strictly in order.
+  __device__ __forceinline__ void slot(int pos, int& j, bool& is_v) const {
+    if (pos == 0) {
+      j = 0;
+      is_v = false;
+    } else if (pos == 2 * n - 1) {
+      j = n - 1;
+      is_v = true;
+    } else if (pos & 1) {
+      j = (pos + 1) >> 1;
+      is_v = false;
+    } else {
+      j = (pos >> 1) - 1;
+      is_v = true;
+    }
   }
   // Valid keys in the t-th tile that query tile x consumes.
   __device__ __forceinline__ int valid(const WorkItem& w, int x, int t) const {
@@ -428,6 +453,7 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
 template <int D>
 struct Smem {
   uint8_t* q;        // [2][kTileBytes]
+  uint8_t* p;        // [kPBufs][kTileBytes]: P of tiles A, B (d = 128)
   uint8_t* kv;       // [kStages][kTileBytes]
   uint64_t* kv_full;
   uint64_t* kv_empty;
@@ -438,8 +464,6 @@ struct Smem {
   uint64_t* p_full;   // [2]
   uint64_t* pv_done;  // [2]
   uint64_t* drain;    // [2]
-  uint64_t* mufu;     // [2][4]: exponential-phase turns, per query tile and sub-partition
-  uint64_t* iturn;    // [2]: MMA-batch issue turns, per query tile
   uint64_t* itq_full;   // [kItemQ]
   uint64_t* itq_empty;  // [kItemQ]
   volatile int* itq;    // [kItemQ] work-item indices handed from the producer to the others
@@ -502,25 +526,24 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
       ++qcnt[x];
     }
     const Stream st(w);
-    for (int j = 0; ok && j < st.n; ++j) {
-      int mask, row0;
-      bool from_cache;
+    for (int pos = 0; ok && pos < 2 * st.n; ++pos) {
+      int j, mask, row0;
+      bool is_v, from_cache;
+      st.slot(pos, j, is_v);
       st.tile(w, j, mask, from_cache, row0);
-      for (int kv = 0; kv < 2; ++kv) {
-        const uint32_t s = ring % C::kStages, ph = (ring / C::kStages) & 1;
-        ok = wait_bar(sm.kv_empty + s, ph ^ 1, ctl);
-        if (!ok) break;
-        if (lane == 0) {
-          const CUtensorMap* m = from_cache ? (kv ? &p.tm_vc : &p.tm_kc) : (kv ? &p.tm_vs : &p.tm_ks);
-          mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
+      const uint32_t s = ring % C::kStages, ph = (ring / C::kStages) & 1;
+      ok = wait_bar(sm.kv_empty + s, ph ^ 1, ctl);
+      if (!ok) break;
+      if (lane == 0) {
+        const CUtensorMap* m = from_cache ? (is_v ? &p.tm_vc : &p.tm_kc) : (is_v ? &p.tm_vs : &p.tm_ks);
+        mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
 #pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, w.head * D + pn * 64, row0,
-                        sm.kv_full + s);
-        }
-        __syncwarp();
-        ++ring;
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, w.head * D + pn * 64, row0,
+                      sm.kv_full + s);
       }
+      __syncwarp();
+      ++ring;
     }
   }
   if (!ok && lane == 0) {
@@ -539,11 +562,17 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
 // tcgen05.commit tracks only the committing thread's MMAs, so every K/V slot is released by
 // two arrivals, one per issuer: a commit after its MMAs read the slot, or, for a tile this
 // query tile does not read, a plain arrive once the tile has landed.
+//
+// Each issuer walks the ring positions in order (K0, K1, V0, K2, V1, ...): S of key tile j+1
+// waits only for the softmax to have read S of tile j (S has its own TMEM columns), so it is
+// computed while that softmax runs; PV of tile j waits for its P.  Because every wait is on
+// the issuer's current ring position or on its own softmax, which only needs earlier
+// positions, no ring depth can deadlock.
 template <int D>
 __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, uint32_t tmem, int X) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0, iturns = 0;
+  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
   bool ok = true;
   int tn = 0;
   (void)tn;
@@ -551,15 +580,10 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
   // Descriptors are computed once; per instruction only a constant is added to the start
   // address field (addresses stay below 256 KiB, so the 14-bit field never carries).
   const uint64_t qdesc = sdesc_sw128(smem_u32(sm.q) + X * C::kTileBytes, 16, 1024);
+  const uint64_t pdesc = sdesc_sw128(smem_u32(sm.p) + X * C::kTileBytes, 16, 1024);
   const uint64_t kdesc0 = sdesc_sw128(smem_u32(sm.kv), 16, 1024);
   const uint64_t vdesc0 = sdesc_sw128(smem_u32(sm.kv), C::kPanelBytes, 1024);
   const uint32_t s_t = tmem + C::s_col(X), o_t = tmem + C::o_col(X), p_t = tmem + C::p_col(X);
-
-  auto release_unread = [&](uint32_t r) {
-    ok = wait_bar(sm.kv_full + r % C::kStages, (r / C::kStages) & 1, ctl);
-    if (ok && lane == 0) mbar_arrive(sm.kv_empty + r % C::kStages);
-    __syncwarp();
-  };
 
   uint32_t kq = 0;
   while (ok) {
@@ -569,73 +593,35 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
     const Stream st(w);
     const uint32_t ring0 = ring;
     ring += 2u * st.n;
-    if (X >= w.n_q) {
-      for (uint32_t r = ring0; ok && r < ring; ++r) release_unread(r);
-      continue;
-    }
-    int s_left = st.count(X);
-    // While both query tiles have a key tile at the same position, their MMA batches
-    // [PV of the previous tile, S of this tile] alternate A, B through an issue token, so the
-    // S that unblocks one tile's next softmax is not interleaved with the other tile's PV.
-    const int paired = (kIssueToken && w.n_q == 2) ? min(st.count(0), st.count(1)) : 0;
-    int t = 0;
+    const bool mine = X < w.n_q;
+    int s_left = mine ? st.count(X) : 0;
     bool first_s = true, first_pv = true;
-    int pend = -1;   // key tile whose PV is still to be issued
-
-    // Waits for the PV of key tile jp: its V tile landed and its P is in TMEM.
-    auto wait_pv = [&](int jp) {
-      BAT_TRACE_EV(1 + X, tn, 3, X, jp);
-      const uint32_t rv = ring0 + 2u * jp + 1;
-      ok = wait_bar(sm.kv_full + rv % C::kStages, (rv / C::kStages) & 1, ctl);
-      if (ok) ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
-      ++p_seen;
-    };
-    // PV of key tile jp (lane 0): O += P . V, P read from TMEM, V (MN-major) from the ring.
-    auto emit_pv = [&](int jp) {
-      const uint32_t s = (ring0 + 2u * jp + 1) % C::kStages;
-      const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
-      // 16 keys = two 8-row swizzle groups (2 KiB); LBO steps between 64-column panels.
-      mma_ts_w(o_t, p_t, vd, C::kIdescPV, first_pv ? 0u : 1u);
-#pragma unroll
-      for (int kk = 1; kk < kTileN / 16; ++kk)
-        mma_ts_w(o_t, p_t + kk * 8, vd + (uint64_t)(kk * 2048 / 16), C::kIdescPV, 1u);
-      tc_commit_w(sm.pv_done + X);
-      tc_commit_w(sm.kv_empty + s);
-    };
-
-    for (int j = 0; ok && j < st.n; ++j) {
-      int mask, row0;
-      bool from_cache;
+    for (int pos = 0; ok && pos < 2 * st.n; ++pos) {
+      int j, mask, row0;
+      bool is_v, from_cache;
+      st.slot(pos, j, is_v);
       st.tile(w, j, mask, from_cache, row0);
-      const uint32_t rk = ring0 + 2u * j, ks = rk % C::kStages;
-      if (!((mask >> X) & 1)) {
-        release_unread(rk);
-        if (ok) release_unread(rk + 1);
+      const uint32_t r = ring0 + pos, s = r % C::kStages;
+      ok = wait_bar(sm.kv_full + s, (r / C::kStages) & 1, ctl);
+      if (!ok) break;
+      if (!mine || !((mask >> X) & 1)) {
+        // A tile this query tile does not read: release the slot once it has landed.
+        if (lane == 0) mbar_arrive(sm.kv_empty + s);
+        __syncwarp();
         continue;
       }
-      if (C::kAliasP && pend >= 0) wait_pv(pend);
-      BAT_TRACE_EV(1 + X, tn, 4, X, s_issued);
-      if (ok) ok = wait_bar(sm.kv_full + ks, (rk / C::kStages) & 1, ctl);
-      if (ok && first_s) {
-        ok = wait_bar(sm.q_full + X, qcnt & 1, ctl);
-        ++qcnt;
-        first_s = false;
-      }
-      // Separate P columns (d = 64): S may be overwritten once the softmax has read the
-      // previous S.  Aliased P (d = 128): this S overwrites the columns the PV issued just
-      // before it reads P from; tcgen05.mma instructions issued by one thread execute in
-      // issue order, so that PV has read its A operand before this S writes its accumulator
-      // (the rule NVIDIA's CUTLASS Blackwell attention mainloop relies on as well).
-      if (ok && !C::kAliasP && s_issued > 0) ok = wait_bar(sm.s_free + X, (s_issued - 1) & 1, ctl);
-      if (ok && t < paired) {
-        ok = wait_bar(sm.iturn + X, (iturns & 1) ^ (X == 0 ? 1u : 0u), ctl);
-        ++iturns;
-      }
-      if (!ok) break;
-      tc_fence_after();
-      if (C::kAliasP && pend >= 0) emit_pv(pend);
-      {
-        const uint64_t kd = kdesc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
+      if (!is_v) {
+        BAT_TRACE_EV(1 + X, tn, 4, X, s_issued);
+        if (first_s) {
+          ok = wait_bar(sm.q_full + X, qcnt & 1, ctl);
+          ++qcnt;
+          first_s = false;
+        }
+        // The softmax must have read the previous S out of these columns.
+        if (ok && s_issued > 0) ok = wait_bar(sm.s_free + X, (s_issued - 1) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t kd = kdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
@@ -643,38 +629,36 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         }
         tc_commit_w(sm.s_full + X);
         if (s_left == 1) tc_commit_w(sm.q_empty + X);
-        tc_commit_w(sm.kv_empty + ks);
-        if (t < paired) mbar_arrive_w(sm.iturn + (1 - X));
+        tc_commit_w(sm.kv_empty + s);
+        --s_left;
+        ++s_issued;
+        BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
+      } else {
+        BAT_TRACE_EV(1 + X, tn, 3, X, p_seen);
+        ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
+        ++p_seen;
+        if (!ok) break;
+        tc_fence_after();
+        // O += P . V: 16 keys per instruction = two 8-row swizzle groups of V (2 KiB); LBO
+        // steps between V's 64-column panels.
+        const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk) {
+          const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
+          const uint64_t vk = vd + (uint64_t)(kk * 2048 / 16);
+          if constexpr (C::kPSmem) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
+            mma_ss_w(o_t, pdesc + off, vk, C::kIdescPV, acc);
+          } else {
+            mma_ts_w(o_t, p_t + kk * 8, vk, C::kIdescPV, acc);
+          }
+        }
+        tc_commit_w(sm.pv_done + X);
+        tc_commit_w(sm.kv_empty + s);
+        first_pv = false;
+        BAT_TRACE_EV(1 + X, tn, 1, X, p_seen);
       }
       __syncwarp();
-      if (!C::kAliasP && pend >= 0) {
-        // Separate P columns: S of this tile went first (the softmax had read the previous S),
-        // so it is computed while the softmax still works on the previous tile; the previous
-        // tile's PV follows as soon as its P is written.
-        wait_pv(pend);
-        if (!ok) break;
-        tc_fence_after();
-        emit_pv(pend);
-        __syncwarp();
-      }
-      if (pend >= 0) first_pv = false;
-      BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
-      --s_left;
-      ++s_issued;
-      ++t;
-      pend = j;
-      if (s_left == 0) {
-        // Exhausted: issue the last PV now, so its V slot is not held while the other query
-        // tile walks the rest of the item.
-        wait_pv(pend);
-        if (!ok) break;
-        tc_fence_after();
-        emit_pv(pend);
-        __syncwarp();
-        first_pv = false;
-        BAT_TRACE_EV(1 + X, tn, 1, X, pend);
-        pend = -1;
-      }
     }
   }
   // Wait for every MMA this warp issued before the CTA frees TMEM.
@@ -694,13 +678,10 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
   const uint32_t tP = tmem + C::p_col(X) + lane_off;
   const uint32_t tO = tmem + C::o_col(X) + lane_off;
   const float sl2 = p.scale_log2;
-  // Warp i of tile A and warp i of tile B run on the same sub-partition and share its MUFU:
-  // while both have a tile at the same position they take turns on the exponentials (A first),
-  // so each runs at the MUFU's full rate while the other waits on its MMAs.
-  const int wq = (threadIdx.x >> 5) & 3;
-  uint64_t* const my_turn = sm.mufu + X * 4 + wq;
-  uint64_t* const other_turn = sm.mufu + (1 - X) * 4 + wq;
-  uint32_t turns = 0;
+  // d = 128: this thread's row of the P tile in shared memory (K-major, 128-byte swizzle:
+  // 16-byte chunk c of row r sits at r * 128 + ((c ^ (r & 7)) << 4) within its 64-key panel).
+  const uint32_t p_row = smem_u32(sm.p) + X * C::kTileBytes + row * 128;
+  const uint32_t p_sw = row & 7;
   uint32_t s_seen = 0, pv_base = 0;
   bool ok = true;
   int tn = 0;
@@ -714,7 +695,6 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     if (X >= w.n_q) continue;
     const Stream st(w);
     const int nX = st.count(X);
-    const int paired = (kMufuTurns && w.n_q == 2) ? min(st.count(0), st.count(1)) : 0;
     float m = -INFINITY, l = 0.f;
     for (int t = 0; t < nX; ++t) {
       const int valid = st.valid(w, X, t);
@@ -726,10 +706,9 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       float s[128];
       tmem_ld128f(tS, s);
       BAT_TRACE_EV(3 + X, tn, 7, X, s_seen);
-      if (!C::kAliasP) {
-        tc_fence_before();
-        mbar_arrive(sm.s_free + X);
-      }
+      // S is in registers: the issuer may compute the next S into these columns.
+      tc_fence_before();
+      mbar_arrive(sm.s_free + X);
       if (valid < kTileN) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = c < valid ? s[c] : -INFINITY;
@@ -767,17 +746,12 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       }
       m = m_new;
       BAT_TRACE_EV(3 + X, tn, 8, X, s_seen);
-      if (t < paired) {
-        ok = wait_bar(my_turn, (turns & 1) ^ (X == 0 ? 1u : 0u), ctl);
-        if (!ok) break;
-        ++turns;
-      }
-      BAT_TRACE_EV(3 + X, tn, 9, X, s_seen);
       const float nm = -m;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
-      // stored to TMEM (asynchronously) while the next half's exponentials run.  Of every eight
-      // columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the MUFU.
+      // stored (TMEM or shared memory, asynchronously) while the next half's exponentials run.
+      // Of every eight columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the
+      // MUFU.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -785,23 +759,16 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
 #pragma unroll
           for (int k = 0; k < 8; k += 2) ffma2(s[c + k], s[c + k + 1], s[c + k], s[c + k + 1], sl2, nm);
 #pragma unroll
-          for (int k = 0; k < 8 - 2 * kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
+          for (int k = 0; k < 8 - 2 * C::kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
 #pragma unroll
-          for (int k = 8 - 2 * kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
+          for (int k = 8 - 2 * C::kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
           fadd2(a0, a1, s[c], s[c + 1]);
           fadd2(a2, a3, s[c + 2], s[c + 3]);
           fadd2(a0, a1, s[c + 4], s[c + 5]);
           fadd2(a2, a3, s[c + 6], s[c + 7]);
         }
-        if (h == 1) {
-          BAT_TRACE_EV(3 + X, tn, 10, X, s_seen);
-          if (t < paired) {
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(other_turn);
-          }
-        }
-        if (!C::kAliasP && t > 0 && h == 0) {
-          // Separate P columns: the previous P must have been consumed before it is overwritten.
+        if (t > 0 && h == 0) {
+          // The previous P must have been consumed before it is overwritten.
           ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
           if (!ok) break;
           tc_fence_after();
@@ -809,12 +776,25 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]);
-        tmem_st32(tP + 32 * h, pk);
+        if constexpr (C::kPSmem) {
+          // Keys 64h .. 64h+63 are panel h of the P tile.
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            st_shared_v4(p_row + h * C::kPanelBytes + ((cc ^ p_sw) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
+                         pk[4 * cc + 3]);
+        } else {
+          tmem_st32(tP + 32 * h, pk);
+        }
       }
       if (!ok) break;
       l += (a0 + a1) + (a2 + a3);
-      tmem_st_wait();
-      tc_fence_before();
+      if constexpr (C::kPSmem) {
+        // Make the generic-proxy stores of P visible to the tensor core (async proxy).
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      } else {
+        tmem_st_wait();
+        tc_fence_before();
+      }
       mbar_arrive(sm.p_full + X);
       BAT_TRACE_EV(3 + X, tn, 2, X, s_seen);
     }
@@ -874,7 +854,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem<D> sm;
   sm.q = base;
-  sm.kv = base + 2 * C::kTileBytes;
+  sm.p = base + 2 * C::kTileBytes;
+  sm.kv = sm.p + C::kPBufs * C::kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm.kv + C::kStages * C::kTileBytes);
   sm.kv_full = bars;
   sm.kv_empty = bars + C::kStages;
@@ -885,9 +866,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.p_full = sm.s_free + 2;
   sm.pv_done = sm.p_full + 2;
   sm.drain = sm.pv_done + 2;
-  sm.mufu = sm.drain + 2;
-  sm.iturn = sm.mufu + 8;
-  sm.itq_full = sm.iturn + 2;
+  sm.itq_full = sm.drain + 2;
   sm.itq_empty = sm.itq_full + kItemQ;
   sm.itq = reinterpret_cast<volatile int*>(sm.itq_empty + kItemQ);
   sm.tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(sm.itq) + kItemQ);
@@ -909,9 +888,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     }
     mbar_init(sm.drain, 1);
     mbar_init(sm.drain + 1, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(sm.mufu + i, 1);
-    mbar_init(sm.iturn, 1);
-    mbar_init(sm.iturn + 1, 1);
     for (int i = 0; i < kItemQ; ++i) {
       mbar_init(sm.itq_full + i, 1);
       mbar_init(sm.itq_empty + i, kItemConsumers);
