@@ -335,6 +335,10 @@ struct Cfg {
   static constexpr bool kPSmem = D == 128;                // P in shared memory (TMEM is full)
   static constexpr int kPBufs = kPSmem ? 2 : 0;            // P tiles in shared memory
   static constexpr int kStages = D == 128 ? 3 : 12;        // K/V ring depth (fills 227 KB)
+  // d = 64: PV is issued in two halves of 64 keys, each as soon as the softmax has written that
+  // half of P, so the next tile's P can overwrite the first half early (measured faster at
+  // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
+  static constexpr int kPVHalves = D == 64 ? 2 : 1;
   // Of every 8 score columns, pairs exponentiated on the FMA pipe (the rest on the MUFU): at
   // d = 64 the MUFU is the busier unit (its exponentials take twice the MMA time).
   static constexpr int kFmaExpPairs = kFmaExpPairsSet >= 0 ? kFmaExpPairsSet : (D == 64 ? 1 : 0);
@@ -344,7 +348,7 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t p_col(int x) { return 384u + 64u * x; }   // d = 64 only
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 6 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 4 + 4 * 2 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kPBufs + kStages) * kTileBytes + kBarBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -461,8 +465,8 @@ struct Smem {
   uint64_t* q_empty;  // [2]
   uint64_t* s_full;   // [2]
   uint64_t* s_free;   // [2]
-  uint64_t* p_full;   // [2]
-  uint64_t* pv_done;  // [2]
+  uint64_t* p_full;   // [2][2]: P of tile x, keys 64h .. 64h+63 written
+  uint64_t* pv_done;  // [2][2]: PV of tile x over keys 64h .. 64h+63 done
   uint64_t* drain;    // [2]
   uint64_t* itq_full;   // [kItemQ]
   uint64_t* itq_empty;  // [kItemQ]
@@ -634,29 +638,35 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         ++s_issued;
         BAT_TRACE_EV(1 + X, tn, 2, X, s_issued);
       } else {
-        BAT_TRACE_EV(1 + X, tn, 3, X, p_seen);
-        ok = wait_bar(sm.p_full + X, p_seen & 1, ctl);
-        ++p_seen;
-        if (!ok) break;
-        tc_fence_after();
-        // O += P . V: 16 keys per instruction = two 8-row swizzle groups of V (2 KiB); LBO
+        // O += P . V of key tile j, in kPVHalves parts (the part over keys 64h .. 64h+63 once the
+        // softmax has written that half of P; with one part, the barriers of half 1 stand for
+        // the whole tile).  16 keys per instruction = two 8-row swizzle groups of V (2 KiB); LBO
         // steps between V's 64-column panels.
         const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk) {
-          const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
-          const uint64_t vk = vd + (uint64_t)(kk * 2048 / 16);
-          if constexpr (C::kPSmem) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
-            mma_ss_w(o_t, pdesc + off, vk, C::kIdescPV, acc);
-          } else {
-            mma_ts_w(o_t, p_t + kk * 8, vk, C::kIdescPV, acc);
+        for (int h = 2 - C::kPVHalves; h < 2; ++h) {
+          BAT_TRACE_EV(1 + X, tn, 3, X, p_seen);
+          ok = wait_bar(sm.p_full + 2 * X + h, p_seen & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = C::kPVHalves == 2 ? 4 * h : 0; kk < 4 * h + 4; ++kk) {
+            const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
+            const uint64_t vk = vd + (uint64_t)(kk * 2048 / 16);
+            if constexpr (C::kPSmem) {
+              const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
+              mma_ss_w(o_t, pdesc + off, vk, C::kIdescPV, acc);
+            } else {
+              mma_ts_w(o_t, p_t + kk * 8, vk, C::kIdescPV, acc);
+            }
           }
+          tc_commit_w(sm.pv_done + 2 * X + h);
+          BAT_TRACE_EV(1 + X, tn, 1, X, p_seen);
         }
-        tc_commit_w(sm.pv_done + X);
+        if (!ok) break;
+        ++p_seen;
         tc_commit_w(sm.kv_empty + s);
         first_pv = false;
-        BAT_TRACE_EV(1 + X, tn, 1, X, p_seen);
       }
       __syncwarp();
     }
@@ -729,7 +739,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       const bool resc = t > 0 && m_new != m;
       if (__any_sync(0xffffffffu, resc)) {
         // O holds the previous tiles' sum: wait for the last PV, then rescale in place.
-        ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
+        ok = wait_bar(sm.pv_done + 2 * X + 1, (pv_base + t - 1) & 1, ctl);
         if (!ok) break;
         tc_fence_after();
         const float alpha = resc ? ex2(m - m_new) : 1.f;
@@ -767,11 +777,14 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
           fadd2(a0, a1, s[c + 4], s[c + 5]);
           fadd2(a2, a3, s[c + 6], s[c + 7]);
         }
-        if (t > 0 && h == 0) {
-          // The previous P must have been consumed before it is overwritten.
-          ok = wait_bar(sm.pv_done + X, (pv_base + t - 1) & 1, ctl);
+        if (t > 0 && (C::kPVHalves == 2 || h == 0)) {
+          // This half of the previous P (with one PV part: all of it) must have been consumed
+          // before it is overwritten.
+          BAT_TRACE_EV(3 + X, tn, 12, X, s_seen);
+          ok = wait_bar(sm.pv_done + 2 * X + (C::kPVHalves == 2 ? h : 1), (pv_base + t - 1) & 1, ctl);
           if (!ok) break;
           tc_fence_after();
+          BAT_TRACE_EV(3 + X, tn, 11, X, s_seen);
         }
         uint32_t pk[32];
 #pragma unroll
@@ -785,23 +798,25 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
         } else {
           tmem_st32(tP + 32 * h, pk);
         }
+        if (C::kPVHalves == 2 || h == 1) {
+          if constexpr (C::kPSmem) {
+            // Make the generic-proxy stores visible to the tensor core (async proxy).
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          } else {
+            tmem_st_wait();
+            tc_fence_before();
+          }
+          mbar_arrive(sm.p_full + 2 * X + h);
+        }
       }
       if (!ok) break;
       l += (a0 + a1) + (a2 + a3);
-      if constexpr (C::kPSmem) {
-        // Make the generic-proxy stores of P visible to the tensor core (async proxy).
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      } else {
-        tmem_st_wait();
-        tc_fence_before();
-      }
-      mbar_arrive(sm.p_full + X);
       BAT_TRACE_EV(3 + X, tn, 2, X, s_seen);
     }
     if (!ok) break;
     // Epilogue: O / l, 16-byte stores of this thread's row.
     BAT_TRACE_EV(3 + X, tn, 5, X, s_seen);
-    ok = wait_bar(sm.pv_done + X, (pv_base + nX - 1) & 1, ctl);
+    ok = wait_bar(sm.pv_done + 2 * X + 1, (pv_base + nX - 1) & 1, ctl);
     if (!ok) break;
     tc_fence_after();
     pv_base += nX;
@@ -864,8 +879,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.s_full = sm.q_empty + 2;
   sm.s_free = sm.s_full + 2;
   sm.p_full = sm.s_free + 2;
-  sm.pv_done = sm.p_full + 2;
-  sm.drain = sm.pv_done + 2;
+  sm.pv_done = sm.p_full + 4;
+  sm.drain = sm.pv_done + 4;
   sm.itq_full = sm.drain + 2;
   sm.itq_empty = sm.itq_full + kItemQ;
   sm.itq = reinterpret_cast<volatile int*>(sm.itq_empty + kItemQ);
@@ -883,8 +898,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
       mbar_init(sm.q_empty + x, 1);
       mbar_init(sm.s_full + x, 1);
       mbar_init(sm.s_free + x, 128);
-      mbar_init(sm.p_full + x, 128);
-      mbar_init(sm.pv_done + x, 1);
+      mbar_init(sm.p_full + 2 * x, 128);
+      mbar_init(sm.p_full + 2 * x + 1, 128);
+      mbar_init(sm.pv_done + 2 * x, 1);
+      mbar_init(sm.pv_done + 2 * x + 1, 1);
     }
     mbar_init(sm.drain, 1);
     mbar_init(sm.drain + 1, 1);
