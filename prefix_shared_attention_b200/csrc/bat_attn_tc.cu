@@ -499,6 +499,9 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
   const int lane = threadIdx.x & 31;
   uint32_t ring = 0, qcnt[2] = {0, 0}, kq = 0;
   bool ok = true;
+  int tn = 0;
+  (void)tn;
+  BAT_TRACE_INIT(0);
   while (ok) {
     const uint32_t slot = kq % kItemQ;
     ok = wait_bar(sm.itq_empty + slot, ((kq / kItemQ) & 1) ^ 1, ctl);
@@ -515,9 +518,11 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
     ++kq;
     if (done) break;
     const WorkItem w = p.items[it];
+    BAT_TRACE_EV(0, tn, 1, 0, kq);
     for (int x = 0; ok && x < w.n_q; ++x) {
       ok = wait_bar(sm.q_empty + x, (qcnt[x] & 1) ^ 1, ctl);
       if (!ok) break;
+      BAT_TRACE_EV(0, tn, 2, x, kq);
       if (lane == 0) {
         mbar_expect_tx(sm.q_full + x, C::kTileBytes);
         const int row0 = x ? w.qB_row0 : w.qA_row0;
@@ -538,6 +543,7 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
       const uint32_t s = ring % C::kStages, ph = (ring / C::kStages) & 1;
       ok = wait_bar(sm.kv_empty + s, ph ^ 1, ctl);
       if (!ok) break;
+      if (pos < 2 || pos == 2 * st.n - 1) BAT_TRACE_EV(0, tn, 3 + (pos == 2 * st.n - 1 ? 2 : pos), 0, kq);
       if (lane == 0) {
         const CUtensorMap* m = from_cache ? (is_v ? &p.tm_vc : &p.tm_kc) : (is_v ? &p.tm_vs : &p.tm_ks);
         mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
@@ -606,6 +612,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       st.slot(pos, j, is_v);
       st.tile(w, j, mask, from_cache, row0);
       const uint32_t r = ring0 + pos, s = r % C::kStages;
+      if (pos == 0) BAT_TRACE_EV(1 + X, tn, 6, X, s_issued);
       ok = wait_bar(sm.kv_full + s, (r / C::kStages) & 1, ctl);
       if (!ok) break;
       if (!mine || !((mask >> X) & 1)) {
@@ -620,6 +627,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
           ok = wait_bar(sm.q_full + X, qcnt & 1, ctl);
           ++qcnt;
           first_s = false;
+          BAT_TRACE_EV(1 + X, tn, 7, X, s_issued);
         }
         // The softmax must have read the previous S out of these columns.
         if (ok && s_issued > 0) ok = wait_bar(sm.s_free + X, (s_issued - 1) & 1, ctl);
