@@ -73,14 +73,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a bf16 [T, H*d] row-major tensor: box 64 columns (128 bytes) x 128 rows,
+// 2-D map over a bf16 [T, H*d] row-major tensor: box 64 columns (128 bytes) x box_rows rows,
 // 128-byte swizzle, zero fill outside the tensor.
-bat_status encode_map(CUtensorMap* m, const void* base, int64_t T, int32_t H, int32_t d, const char* name) {
+bat_status encode_map(CUtensorMap* m, const void* base, int64_t T, int32_t H, int32_t d, const char* name,
+                      uint32_t box_rows = bat::kTileN) {
   auto fn = encode_fn();
   if (!fn) return fail(BAT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {(cuuint64_t)H * d, (cuuint64_t)(T > 0 ? T : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)H * d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)bat::kTileN};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -338,6 +339,9 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
     if ((st = encode_map(&p.tm_vc, has_cache ? v_cache : v_suf, has_cache ? plan->T_cache : plan->T_suf, plan->H,
                          plan->d, "v_cache")) != BAT_OK)
       return st;
+    // The output map stores one warp's 32 rows at a time (rows of a partial query tile that
+    // belong to another request are never covered: such warps store row by row instead).
+    if ((st = encode_map(&p.tm_o, out, plan->T_suf, plan->H, plan->d, "out", 32)) != BAT_OK) return st;
     p.items = plan->d_items;
     p.n_items = plan->host.n_items;
     p.out = out;

@@ -139,6 +139,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Shared -> global tensor store (bulk group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The issuing thread's bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The issuing thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -700,6 +713,9 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
   // 16-byte chunk c of row r sits at r * 128 + ((c ^ (r & 7)) << 4) within its 64-key panel).
   const uint32_t p_row = smem_u32(sm.p) + X * C::kTileBytes + row * 128;
   const uint32_t p_sw = row & 7;
+  const int wq = (threadIdx.x >> 5) & 3;           // this warp's 32-row group of the tile
+  const uint32_t lane = threadIdx.x & 31;
+  bool o_pending = false;                          // lane 0: a bulk store still reads this warp's P rows
   uint32_t s_seen = 0, pv_base = 0;
   bool ok = true;
   int tn = 0;
@@ -709,8 +725,19 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
   while (ok) {
     const int it = pop_item<D>(sm, kq, ctl, ok);
     if (it < 0) break;
+    BAT_TRACE_EV(3 + X, tn, 15, X, s_seen);
     const WorkItem w = p.items[it];
     if (X >= w.n_q) continue;
+    BAT_TRACE_EV(3 + X, tn, 16, X, s_seen);
+    if constexpr (C::kPSmem) {
+      if (o_pending) {
+        // The previous item's output leaves this warp's P rows by a bulk store: it must have
+        // read them before this item's P overwrites them.
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+        o_pending = false;
+      }
+    }
     const Stream st(w);
     const int nX = st.count(X);
     float m = -INFINITY, l = 0.f;
@@ -827,13 +854,49 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     ok = wait_bar(sm.pv_done + 2 * X + 1, (pv_base + nX - 1) & 1, ctl);
     if (!ok) break;
     tc_fence_after();
+    BAT_TRACE_EV(3 + X, tn, 13, X, s_seen);
     pv_base += nX;
     const int rows = X ? w.qB_rows : w.qA_rows;
     const int qrow = (X ? w.qB_row0 : w.qA_row0) + row;
     const bool live = row < rows;
     const float inv = 1.f / l;
     const float lse2 = m + __log2f(l);
-    if (w.split_slot < 0) {
+    bool o_stored = false;
+    if constexpr (C::kPSmem) {
+      if (w.split_slot < 0 && rows >= 32 * (wq + 1)) {
+        // All 32 rows of this warp belong to the request: O / l goes into the warp's rows of the
+        // (now free) P tile in the 128-byte-swizzled layout, then one bulk tensor store per
+        // 64-column panel writes them out, fully coalesced.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_shared_v4(p_row + (c >> 1) * C::kPanelBytes + (((uint32_t)((c & 1) * 4 + i) ^ p_sw) << 4), pk[4 * i],
+                         pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          const int y = (X ? w.qB_row0 : w.qA_row0) + 32 * wq;
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_store_2d(&p.tm_o, sm.p + X * C::kTileBytes + pn * C::kPanelBytes + wq * 32 * 128, w.head * D + pn * 64, y);
+          bulk_commit();
+        }
+        o_pending = true;
+        BAT_TRACE_EV(3 + X, tn, 14, X, s_seen);
+        if (p.lse) p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
+        o_stored = true;
+      }
+    }
+    if (o_stored) {
+    } else if (w.split_slot < 0) {
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)qrow * p.H + w.head) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -849,6 +912,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
+      BAT_TRACE_EV(3 + X, tn, 14, X, s_seen);
       if (live && p.lse) p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
     } else {
       const int64_t slot = w.split_slot + X;
@@ -867,6 +931,11 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       }
       if (live) p.part_lse[slot * kTileM + row] = lse2;
     }
+  }
+  if constexpr (C::kPSmem) {
+    // Bulk stores must be complete (and done reading shared memory) before the CTA exits.
+    if (o_pending && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 }
 
@@ -926,6 +995,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     prefetch_tmap(&p.tm_vs);
     prefetch_tmap(&p.tm_kc);
     prefetch_tmap(&p.tm_vc);
+    prefetch_tmap(&p.tm_o);
   }
   if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sm.tmem_slot)),

@@ -11,6 +11,7 @@ namespace bat {
 // Tensor-core path (bf16 in, fp32 accumulate), d in {64, 128}.
 struct alignas(64) TcParams {
   CUtensorMap tm_q, tm_ks, tm_vs, tm_kc, tm_vc;  // [T, H*d] 2-D maps, box 64 x 128, 128B swizzle
+  CUtensorMap tm_o;     // output [T_suf, H*d], box 64 x 32 (one warp's rows), 128B swizzle
   const WorkItem* items;
   int64_t n_items;
   void* out;            // bf16 [T_suf, H, d]
