@@ -336,7 +336,11 @@ def main():
     req_s = tab.R * world * args.steps / (elapsed_ms * 1e-3)
     peaks, peak_kind = load_peaks()
     achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    # The denominator follows how long the kernel holds the tensor pipe: a timed region of a
+    # second or more runs under the board's power cap like the sustained GEMM measurement
+    # (seconds back to back), a shorter one is compared with the burst figure.
+    sustained = elapsed_ms >= 1000.0 and "bf16_tflops_sustained" in peaks
+    peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
     kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
     traffic = traffic_per_launch(args.workload, kernel_src)
 
@@ -410,7 +414,9 @@ def main():
             "requests_per_s": req_s,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                         "peak_source": f"{peak_kind} " + ("bf16_tflops_sustained (timed region %.1f s under the power cap)"
+                                                           % (elapsed_ms / 1e3) if sustained else "bf16_tflops (burst)"),
+                         "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "kernel": "bat_attn_tc_kernel", "kernel_ms_per_launch": kernel_ms,
                          "alg_gflop_per_launch": [f / 1e9 for f in flops_l],

@@ -62,9 +62,33 @@ __device__ __forceinline__ void trace(unsigned long long* tp, int& n, uint32_t e
 }
 #define BAT_TRACE_INIT(role) unsigned long long* trace_p = trace_base(role)
 #define BAT_TRACE_EV(role, n, ev, x, idx) trace(trace_p, n, ev, x, idx)
+#define BAT_PHASE_FLUSH() ((void)0)
+#elif defined(BAT_PHASE)
+// Compile-time phase profile (off unless built with -DBAT_PHASE): every warp accumulates, per
+// trace event code, the clocks since its previous event in registers and writes the totals
+// once at the end ([grid][12 warps][20] words), so the profile barely perturbs the timing.
+__device__ unsigned* g_phase;
+#define BAT_TRACE_INIT(role)                                                  \
+  uint32_t ph_acc[20];                                                        \
+  _Pragma("unroll") for (int ph_i = 0; ph_i < 20; ++ph_i) ph_acc[ph_i] = 0; \
+  uint32_t ph_last = (uint32_t)clock64()
+#define BAT_TRACE_EV(role, n, ev, x, idx)      \
+  do {                                         \
+    const uint32_t ph_c = (uint32_t)clock64(); \
+    ph_acc[ev] += ph_c - ph_last;              \
+    ph_last = ph_c;                            \
+  } while (0)
+#define BAT_PHASE_FLUSH()                                                                 \
+  do {                                                                                    \
+    if (g_phase && (threadIdx.x & 31) == 0) {                                             \
+      unsigned* ph_o = g_phase + ((size_t)blockIdx.x * 12 + (threadIdx.x >> 5)) * 20;     \
+      _Pragma("unroll") for (int ph_i = 0; ph_i < 20; ++ph_i) ph_o[ph_i] = ph_acc[ph_i]; \
+    }                                                                                     \
+  } while (0)
 #else
 #define BAT_TRACE_INIT(role) ((void)0)
 #define BAT_TRACE_EV(role, n, ev, x, idx) ((void)0)
+#define BAT_PHASE_FLUSH() ((void)0)
 #endif
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
@@ -569,6 +593,7 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
       ++ring;
     }
   }
+  BAT_PHASE_FLUSH();
   if (!ok && lane == 0) {
     // Let every copy this warp issued land before the CTA releases its shared memory.
     const uint32_t n = ring < (uint32_t)C::kStages ? ring : (uint32_t)C::kStages;
@@ -692,6 +717,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       __syncwarp();
     }
   }
+  BAT_PHASE_FLUSH();
   // Wait for every MMA this warp issued before the CTA frees TMEM.
   if (lane == 0) {
     tc_commit(sm.drain + X);
@@ -932,6 +958,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       if (live) p.part_lse[slot * kTileM + row] = lse2;
     }
   }
+  BAT_PHASE_FLUSH();
   if constexpr (C::kPSmem) {
     // Bulk stores must be complete (and done reading shared memory) before the CTA exits.
     if (o_pending && lane == 0) bulk_wait_all();
@@ -1053,6 +1080,10 @@ cudaError_t launch_attn_tc(int d, const TcParams& p, int grid, cudaStream_t s) {
 #ifdef BAT_TRACE
 extern "C" int bat_debug_set_trace(void* buf) {
   return (int)cudaMemcpyToSymbol(g_trace, &buf, sizeof(buf));
+}
+#elif defined(BAT_PHASE)
+extern "C" int bat_debug_set_phase(void* buf) {
+  return (int)cudaMemcpyToSymbol(g_phase, &buf, sizeof(buf));
 }
 #endif
 
