@@ -370,8 +370,10 @@ struct Cfg {
   static constexpr int kPanelBytes = kTileM * 128;       // 128 rows x 128 bytes
   static constexpr int kTileBytes = kPanels * kPanelBytes;
   static constexpr bool kPSmem = D == 128;                // P in shared memory (TMEM is full)
-  static constexpr int kPBufs = kPSmem ? 2 : 0;            // P tiles in shared memory
-  static constexpr int kStages = D == 128 ? 3 : 12;        // K/V ring depth (fills 227 KB)
+  // One shared-memory tile per query tile: P (d = 128), and at the end of an item the staging
+  // buffer of the output tile (both d).
+  static constexpr int kPBufs = 2;
+  static constexpr int kStages = D == 128 ? 3 : 10;        // K/V ring depth (fills 227 KB)
   // d = 64: PV is issued in two halves of 64 keys, each as soon as the softmax has written that
   // half of P, so the next tile's P can overwrite the first half early (measured faster at
   // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
@@ -494,7 +496,7 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
 template <int D>
 struct Smem {
   uint8_t* q;        // [2][kTileBytes]
-  uint8_t* p;        // [kPBufs][kTileBytes]: P of tiles A, B (d = 128)
+  uint8_t* p;        // [kPBufs][kTileBytes]: P of tiles A, B (d = 128) / output staging
   uint8_t* kv;       // [kStages][kTileBytes]
   uint64_t* kv_full;
   uint64_t* kv_empty;
@@ -755,7 +757,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     const WorkItem w = p.items[it];
     if (X >= w.n_q) continue;
     BAT_TRACE_EV(3 + X, tn, 16, X, s_seen);
-    if constexpr (C::kPSmem) {
+    {
       if (o_pending) {
         // The previous item's output leaves this warp's P rows by a bulk store: it must have
         // read them before this item's P overwrites them.
@@ -888,11 +890,12 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     const float inv = 1.f / l;
     const float lse2 = m + __log2f(l);
     bool o_stored = false;
-    if constexpr (C::kPSmem) {
+    {
       if (w.split_slot < 0 && rows >= 32 * (wq + 1)) {
-        // All 32 rows of this warp belong to the request: O / l goes into the warp's rows of the
-        // (now free) P tile in the 128-byte-swizzled layout, then one bulk tensor store per
-        // 64-column panel writes them out, fully coalesced.
+        // All 32 rows of this warp belong to the request: O / l goes into the warp's rows of its
+        // shared-memory tile (P at d = 128, free after the last PV; a staging tile at d = 64)
+        // in the 128-byte-swizzled layout, then one bulk tensor store per 64-column panel
+        // writes them out, fully coalesced.
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -959,7 +962,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
     }
   }
   BAT_PHASE_FLUSH();
-  if constexpr (C::kPSmem) {
+  {
     // Bulk stores must be complete (and done reading shared memory) before the CTA exits.
     if (o_pending && lane == 0) bulk_wait_all();
     __syncwarp();
