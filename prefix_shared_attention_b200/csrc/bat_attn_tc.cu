@@ -352,9 +352,10 @@ struct Cfg {
   // half of P, so the next tile's P can overwrite the first half early (measured faster at
   // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
   static constexpr int kPVHalves = D == 64 ? 2 : 1;
-  // Of every 8 score columns, pairs exponentiated on the FMA pipe (the rest on the MUFU): at
-  // d = 64 the MUFU is the busier unit (its exponentials take twice the MMA time).
-  static constexpr int kFmaExpPairs = kFmaExpPairsSet >= 0 ? kFmaExpPairsSet : (D == 64 ? 1 : 0);
+  // Of every 8 score columns, pairs exponentiated on the FMA pipe (the rest on the MUFU).
+  // Measured no faster at either d (the exponential phase is not bound by MUFU throughput),
+  // so none by default; -DBAT_FMA_EXP_PAIRS=n selects n.
+  static constexpr int kFmaExpPairs = kFmaExpPairsSet >= 0 ? kFmaExpPairsSet : 0;
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
   __host__ __device__ static constexpr uint32_t o_col(int x) { return 256u + (uint32_t)D * x; }
