@@ -133,11 +133,14 @@ def fits_launches(tab, spec, free_bytes, elt):
 # --------------------------------------------------------------------------------------------
 # CPU oracle (reference arm and cpu_baseline): the fp64 oracle as it stands, on a bounded sample
 
-def oracle_sample(workload, target_s=12.0, seed=99):
+def oracle_sample(workload, target_s=12.0, seed=99, prefix_side=False):
     """Seeded sample of requests (stratified by prefix kind), its host inputs, and its FLOPs."""
     import oracle
     spec = CONFIGS[workload]
     tab = make_table(workload)
+    if prefix_side:
+        from workloads import prefix_side_table
+        tab = prefix_side_table(tab)
     rng = np.random.default_rng(seed)
     order = []
     kinds = np.unique(tab.kind)
@@ -154,8 +157,8 @@ def oracle_sample(workload, target_s=12.0, seed=99):
         remap = np.full(tab.P, -1, np.int64)
         remap[used] = np.arange(len(used))
         from workloads import RequestTable
-        t = RequestTable(tab.prefix_len[used], np.where(sub.req_prefix >= 0, remap[sub.req_prefix], -1),
-                         sub.suffix_len, sub.kind)
+        mapped = remap[np.clip(sub.req_prefix, 0, None)] if tab.P else np.zeros_like(sub.req_prefix)
+        t = RequestTable(tab.prefix_len[used], np.where(sub.req_prefix >= 0, mapped, -1), sub.suffix_len, sub.kind)
         x = host_tensors(t, spec.H, spec.d, spec.dtype, spec.seed + 5)
         x = {k: v.double().numpy() for k, v in x.items()}
         return t, x
@@ -191,14 +194,15 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(workload, target_s=12.0):
-    spec, tab, t, x, run, n = oracle_sample(workload, target_s)
+def cpu_baseline(workload, target_s=12.0, prefix_side=False):
+    spec, tab, t, x, run, n = oracle_sample(workload, target_s, prefix_side=prefix_side)
     flops = workload_flops_bytes(t, spec.H, spec.d, 2)[0]
     s0 = time.perf_counter()
     run(t, x)
     dt = time.perf_counter() - s0
+    what = "prefixes (prefix-side step)" if prefix_side else "requests"
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} of {tab.R} requests of '{workload}' (stratified by prefix kind), fp64 numpy, "
+            "sample": f"{n} of {tab.R} {what} of '{workload}' (stratified by prefix kind), fp64 numpy, "
                       f"{flops / 1e9:.1f} GFLOP in {dt:.2f} s",
             "requests_per_s": n / dt}
 
@@ -206,7 +210,8 @@ def cpu_baseline(workload, target_s=12.0):
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    spec, tab, t, x, run, n = oracle_sample(args.workload, target_s=max(5.0, 150.0 / max(args.steps + args.warmup, 1)))
+    spec, tab, t, x, run, n = oracle_sample(args.workload, target_s=max(5.0, 150.0 / max(args.steps + args.warmup, 1)),
+                                            prefix_side=args.prefix_side)
     flops = workload_flops_bytes(t, spec.H, spec.d, 2)[0]
     for _ in range(args.warmup):
         run(t, x)
@@ -219,7 +224,8 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample_requests": n, "requests": tab.R, "H": spec.H, "d": spec.d},
+            "config": {"workload": args.workload + ("/prefix-side" if args.prefix_side else ""), "sample_requests": n,
+                       "requests": tab.R, "H": spec.H, "d": spec.d},
             "requests_per_s": n * args.steps / dt,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{n} of {tab.R} requests per step, fp64 numpy oracle"},
@@ -242,6 +248,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--launches", type=int, default=0, help="override the number of launches per step")
+    ap.add_argument("--prefix-side", action="store_true",
+                    help="time the prefix-side step instead: every prefix the workload reads attends over "
+                         "its own tokens (the outputs of the prefix tokens themselves)")
     ap.add_argument("--subset", type=int, default=0,
                     help="profiling aid: only the first N requests (and the prefixes they read); not a bench line")
     args = ap.parse_args()
@@ -270,6 +279,9 @@ def main():
     tab = make_table(args.workload)
     if args.subset:
         tab = tab.compact(np.arange(min(args.subset, tab.R)))
+    if args.prefix_side:
+        from workloads import prefix_side_table
+        tab = prefix_side_table(tab)
     free, total = torch.cuda.mem_get_info()
     n_launch = args.launches or fits_launches(tab, spec, free, elt)
     parts = split_launches(tab, n_launch)
@@ -281,7 +293,9 @@ def main():
     suf = device_tensors(parts[0], spec.H, spec.d, spec.dtype, seed + 1, device=dev, which=("q", "k_suf", "v_suf"),
                          rows=rows)
     out = torch.empty_like(suf["q"])
+    t_plan = time.perf_counter()
     plans = [bat.Plan(p.req_prefix, p.suffix_offsets, p.prefix_offsets, spec.H, spec.d, bat.BAT_BF16) for p in parts]
+    plan_ms = (time.perf_counter() - t_plan) * 1e3   # host grouping pass + work-list upload, all launches
     ws_bytes = max(pl.workspace_bytes for pl in plans)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     launches_per_step = sum(1 + (pl.info().n_merges > 0) for pl in plans)
@@ -336,13 +350,16 @@ def main():
     req_s = tab.R * world * args.steps / (elapsed_ms * 1e-3)
     peaks, peak_kind = load_peaks()
     achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
+    # Which roof binds: algorithmic FLOP per byte against the ridge of the measured peaks.
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    hbm_bound = step_flops / step_bytes < ridge
     # The denominator follows how long the kernel holds the tensor pipe: a timed region of a
     # second or more runs under the board's power cap like the sustained GEMM measurement
     # (seconds back to back), a shorter one is compared with the burst figure.
     sustained = elapsed_ms >= 1000.0 and "bf16_tflops_sustained" in peaks
     peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
     kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
-    traffic = traffic_per_launch(args.workload, kernel_src)
+    traffic = None if args.prefix_side else traffic_per_launch(args.workload, kernel_src)
 
     # End to end through the public API with host buffers: per launch, H2D of the request
     # tokens (q, k, v) from pinned memory, the forward, D2H of the output.  The prefix cache is
@@ -400,29 +417,39 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         del suf, cache, out, ws
         torch.cuda.empty_cache()
-        base = cpu_baseline(args.workload)
+        base = cpu_baseline(args.workload, prefix_side=args.prefix_side)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload + (f"[:{args.subset}]" if args.subset else ""), "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
+            "config": {"workload": args.workload + (f"[:{args.subset}]" if args.subset else "")
+                                   + ("/prefix-side" if args.prefix_side else ""), "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
                        "prefixes_cached": tab.P, "tokens_suffix": tab.T_suf, "tokens_cache": tab.T_cache,
                        "l2": "inputs larger than L2 (%.0f GB per launch)" % (step_bytes / n_launch / 1e9),
                        "parallelism": f"dp{world}" if world > 1 else "single"},
             "requests_per_s": req_s,
+            "plan_ms": plan_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} " + ("bf16_tflops_sustained (timed region %.1f s under the power cap)"
                                                            % (elapsed_ms / 1e3) if sustained else "bf16_tflops (burst)"),
                          "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "frac_of_spec": achieved / 2250.0,
+                         "flop_per_byte": step_flops / step_bytes, "ridge_flop_per_byte": ridge,
                          "kernel": "bat_attn_tc_kernel", "kernel_ms_per_launch": kernel_ms,
                          "alg_gflop_per_launch": [f / 1e9 for f in flops_l],
                          "alg_gb_per_launch": [b / 1e9 for b in bytes_l]},
             "cpu_baseline": base, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
         }
+        if hbm_bound:
+            # Left of the ridge: the bandwidth roof binds; report against the measured copy rate.
+            gbs = step_bytes / (sum(kernel_ms) * 1e-3) / 1e9
+            line["roofline"].update({"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                     "frac": gbs / float(peaks["hbm_gbs"]),
+                                     "peak_source": f"{peak_kind} hbm_gbs", "tensor_tflops": achieved})
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

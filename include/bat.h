@@ -108,6 +108,25 @@ bat_status bat_plan_create(const int32_t* req_prefix, const int64_t* suffix_offs
                            int32_t d, bat_dtype dt, const bat_plan_options* opts, void* stream,
                            bat_plan** out);
 
+/*
+ * bat_plan_create_prefix_side - plan for the prefix-side step: the outputs of the prefix
+ * tokens themselves.  Lead page (Bat), section "Problem": the chosen prefix block's K/V is
+ * computed once and cached for every request that reuses it; section "This paper's idea":
+ * the tokens of a block are order-agnostic, so within its own block a token attends with no
+ * mask.  Each prefix's tokens therefore attend over that prefix's tokens only: the forward
+ * with no cached prefix (Lp = 0), the prefix tokens taking the place of a request's own.
+ *   src_offsets  HOST int64 [num_prefixes + 1], non-decreasing: prefix i owns rows
+ *                [so[i], so[i+1]) of the q/k/v tensors later passed to bat_attention_forward
+ *                as q, k_suf, v_suf (k_cache = v_cache = NULL); its outputs land in the same
+ *                rows of `out`.
+ *   H, d, dt, opts, stream, out   as for bat_plan_create
+ * Equivalent to bat_plan_create with req_prefix = -1 for every prefix and P = 0.
+ * Errors: those of bat_plan_create; BAT_ERR_INVALID_ARG for num_prefixes < 0.
+ */
+bat_status bat_plan_create_prefix_side(const int64_t* src_offsets, int32_t num_prefixes, int32_t H,
+                                       int32_t d, bat_dtype dt, const bat_plan_options* opts,
+                                       void* stream, bat_plan** out);
+
 /* Releases the plan and its device work list.  Synchronises the device first (cudaFree),
  * so work already enqueued with the plan completes.  NULL is accepted. */
 bat_status bat_plan_destroy(bat_plan* plan);

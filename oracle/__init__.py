@@ -23,4 +23,5 @@ from .attention import (  # noqa: F401
     bipartite_attention_split,
     merge_partials,
     chunk_partial,
+    prefix_side_attention,
 )

@@ -113,6 +113,38 @@ def bipartite_attention(q, k_suf, v_suf, k_cache, v_cache, prefix_offsets, suffi
     return out, lse
 
 
+def prefix_side_attention(q, k, v, src_offsets, scale: Optional[float] = None,
+                          prefixes: Optional[Iterable[int]] = None):
+    """The prefix tokens' own outputs (the prefix-side step).
+
+    Lead page, section "Problem": the chosen prefix block's K/V is computed once and cached
+    for the requests that reuse it; section "This paper's idea": the tokens of a block are
+    order-agnostic.  Within its own block a prefix token therefore attends, with no mask, over
+    that block's tokens only, per head:
+
+        O_p = softmax_row( scale * Qp . Kp^T ) . Vp
+
+    q, k, v: [T, H, d]; prefix p owns rows [src_offsets[p], src_offsets[p+1]).
+    Returns (out [T, H, d] fp64, lse [H, T] fp64); rows of prefixes not selected are NaN.
+    """
+    q, k, v = map(_as64, (q, k, v))
+    T, H, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    n = len(src_offsets) - 1
+    out = np.full((T, H, v.shape[2]), np.nan)
+    lse = np.full((H, T), np.nan)
+    for p in (range(n) if prefixes is None else prefixes):
+        s0, s1 = int(src_offsets[p]), int(src_offsets[p + 1])
+        if s1 == s0:
+            continue
+        for h in range(H):
+            O, L = attend(q[s0:s1, h, :], k[s0:s1, h, :], v[s0:s1, h, :], scale)
+            out[s0:s1, h, :] = O
+            lse[h, s0:s1] = L
+    return out, lse
+
+
 def merge_partials(parts: Sequence[Tuple[np.ndarray, np.ndarray]]) -> Tuple[np.ndarray, np.ndarray]:
     """Log-sum-exp merge of softmax partials over disjoint key sets.
 

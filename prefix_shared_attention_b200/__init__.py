@@ -29,5 +29,6 @@ from ._bat import (  # noqa: F401
     bat_version,
     exported_symbols,
     last_error,
+    prefix_build,
 )
 from .metrics import algorithmic_bytes, algorithmic_flops  # noqa: F401

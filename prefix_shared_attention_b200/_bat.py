@@ -53,6 +53,7 @@ _SIGNATURES = {
     "bat_prefix_kv_build": (_i32, [_vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "bat_plan_create": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, C.POINTER(PlanOptions), _vp,
                                C.POINTER(_vp)]),
+    "bat_plan_create_prefix_side": (_i32, [_vp, _i32, _i32, _i32, _i32, C.POINTER(PlanOptions), _vp, C.POINTER(_vp)]),
     "bat_plan_destroy": (_i32, [_vp]),
     "bat_plan_info": (_i32, [_vp, C.POINTER(PlanInfo)]),
     "bat_workspace_bytes": (_sz, [_vp]),
@@ -138,6 +139,28 @@ class Plan:
         self.handle = h
         self.H, self.d, self.dtype = H, d, dtype
 
+    @classmethod
+    def prefix_side(cls, src_offsets, H: int, d: int, dtype: int = BAT_BF16, split_mode: int = 0,
+                    split_chunk_tiles: int = 0, num_sms: int = 0, host_only: bool = False, stream=None) -> "Plan":
+        """Plan of the prefix-side step: prefix i's tokens (rows ``src_offsets[i] ..
+        src_offsets[i+1]`` of the q/k/v given to the forward as q, k_suf, v_suf) attend over
+        that prefix's tokens only (no cached prefix)."""
+        self = cls.__new__(cls)
+        so = np.ascontiguousarray(src_offsets, dtype=np.int64)
+        n = int(so.shape[0]) - 1
+        if n < 0:
+            raise BatError(BAT_ERR_INVALID_ARG, "src_offsets needs at least one entry")
+        self._rp = np.full(n, -1, dtype=np.int32)
+        self._so = so
+        self._po = np.zeros(1, dtype=np.int64)
+        opts = PlanOptions(split_mode, split_chunk_tiles, num_sms, 1 if host_only else 0)
+        h = C.c_void_p()
+        st = None if host_only else _stream_handle(stream)
+        check(lib.bat_plan_create_prefix_side(_ptr(so), n, H, d, dtype, C.byref(opts), st, C.byref(h)))
+        self.handle = h
+        self.H, self.d, self.dtype = H, d, dtype
+        return self
+
     def info(self) -> PlanInfo:
         i = PlanInfo()
         check(lib.bat_plan_info(self.handle, C.byref(i)))
@@ -186,6 +209,19 @@ def bat_prefix_kv_build(k_src, v_src, src_offsets, dst_offsets, k_cache, v_cache
     check(lib.bat_prefix_kv_build(k_src.data_ptr(), v_src.data_ptr(), _ptr(so), n, _ptr(do), H, d,
                                   dtype_code(k_src.dtype), k_cache.data_ptr(), v_cache.data_ptr(),
                                   _stream_handle(stream)))
+
+
+def prefix_build(q_src, k_src, v_src, src_offsets, dst_offsets, k_cache, v_cache, out=None, lse=None,
+                 scale: float = 0.0, stream=None):
+    """Prefix-side step for newly cached prefixes: pack their K/V into the pool
+    (bat_prefix_kv_build) and compute the prefix tokens' own outputs (a prefix-side plan and
+    bat_attention_forward).  Tensors are torch device tensors [T, H, d]; returns ``out``
+    (rows of q_src)."""
+    bat_prefix_kv_build(k_src, v_src, src_offsets, dst_offsets, k_cache, v_cache, stream=stream)
+    H, d = int(q_src.shape[1]), int(q_src.shape[2])
+    with Plan.prefix_side(src_offsets, H, d, dtype_code(q_src.dtype), stream=stream) as plan:
+        out = bat_attention_forward(plan, q_src, k_src, v_src, out=out, lse=lse, scale=scale, stream=stream)
+    return out
 
 
 def bat_attention_forward(plan: Plan, q, k_suf, v_suf, k_cache=None, v_cache=None, out=None, lse=None,

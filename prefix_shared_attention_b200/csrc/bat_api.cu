@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <vector>
 #include <mutex>
 #include <string>
 
@@ -229,6 +230,19 @@ bat_status bat_plan_create(const int32_t* req_prefix, const int64_t* suffix_offs
   }
   *out = plan;
   return BAT_OK;
+}
+
+bat_status bat_plan_create_prefix_side(const int64_t* src_offsets, int32_t num_prefixes, int32_t H, int32_t d,
+                                       bat_dtype dt, const bat_plan_options* opts, void* stream, bat_plan** out) {
+  g_err.clear();
+  if (num_prefixes < 0) return fail(BAT_ERR_INVALID_ARG, "num_prefixes=%d < 0", num_prefixes);
+  if (num_prefixes > 0 && !src_offsets) return fail(BAT_ERR_INVALID_ARG, "src_offsets must be non-null");
+  // Every prefix becomes a request with no cached prefix whose own tokens are the prefix's.
+  std::vector<int32_t> req_prefix((size_t)num_prefixes, -1);
+  const int64_t no_cache[1] = {0};
+  const int64_t empty_so[1] = {0};
+  return bat_plan_create(num_prefixes ? req_prefix.data() : nullptr, num_prefixes ? src_offsets : empty_so,
+                         no_cache, num_prefixes, 0, H, d, dt, opts, stream, out);
 }
 
 bat_status bat_plan_destroy(bat_plan* plan) {

@@ -245,3 +245,32 @@ def test_mixed_sampled_one_launch():
     if free < 150e9:
         pytest.skip(f"needs ~140 GB free device memory, {free / 1e9:.0f} GB free")
     sampled_parity("mixed", 24, launch=3, n_launches=8)
+
+
+# --------------------------------------------------------------------------------------
+# prefix-side step: the prefix tokens' own outputs, plus the K/V packed into the pool
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 64), ("bf16", 128), ("fp32", 32)])
+def test_prefix_side_step(dtype, d):
+    lens = [0, 1, 63, 128, 129, 300, 517] if dtype == "bf16" else [0, 1, 40, 129]
+    H = 2
+    tab = RequestTable(np.zeros(0, np.int64), np.full(len(lens), -1), np.array(lens))
+    x = host_tensors(tab, H, d, dtype, 77)
+    q, k, v = (x[n].cuda() for n in ("q", "k_suf", "v_suf"))
+    so = tab.suffix_offsets
+    # Pack into a pool laid out in reverse prefix order (gaps of 3 rows between prefixes).
+    dst, pos = np.zeros(len(lens), np.int64), 0
+    for i in reversed(range(len(lens))):
+        dst[i] = pos
+        pos += lens[i] + 3
+    kc = torch.zeros((pos, H, d), dtype=k.dtype, device="cuda")
+    vc = torch.zeros_like(kc)
+    lse = torch.full((H, max(tab.T_suf, 1)), float("nan"), device="cuda")
+    out = bat.prefix_build(q, k, v, so, dst, kc, vc, lse=lse)
+    assert bat.bat_get_device_status() == bat.BAT_OK, bat.last_error()
+    for i, L in enumerate(lens):
+        assert torch.equal(kc[dst[i]:dst[i] + L], k[so[i]:so[i + 1]]), f"K of prefix {i} not packed exactly"
+        assert torch.equal(vc[dst[i]:dst[i] + L], v[so[i]:so[i + 1]]), f"V of prefix {i} not packed exactly"
+    ref_o, ref_l = oracle.prefix_side_attention(x["q"].double().numpy(), x["k_suf"].double().numpy(),
+                                                x["v_suf"].double().numpy(), so)
+    assert_parity(out, lse, ref_o, ref_l, f"prefix side {dtype} d={d}")

@@ -316,6 +316,58 @@ def test_prefix_of_length_zero_equals_no_prefix():
     np.testing.assert_allclose(la, lb, rtol=0, atol=0)
 
 
+# ----------------------------------------------------------------------------------------
+# prefix-side step: each prefix's tokens attend over that prefix's tokens only
+
+def _prefix_inputs(seed, lens, H=2, d=8):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lens))
+    so = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    x = {k: rng.standard_normal((T, H, d)) for k in ("q", "k", "v")}
+    return so, x
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefix_side_matches_brute_force(seed):
+    lens = [0, 1, 5, 9, 3][seed:] + [7]
+    so, x = _prefix_inputs(seed, lens)
+    o, l = oracle.prefix_side_attention(x["q"], x["k"], x["v"], so)
+    # The element-by-element definition, with every prefix as a request that has no cached
+    # prefix and its own tokens as the suffix.
+    tab = RequestTable(np.zeros(0, np.int64), np.full(len(lens), -1), np.array(lens))
+    empty = x["k"][:0]
+    bo, bl = brute_force(x["q"], x["k"], x["v"], empty, empty, tab.prefix_offsets, so, tab.req_prefix)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l, bl, rtol=1e-12, atol=1e-13)
+
+
+def test_prefix_side_matches_library_attention():
+    import torch
+    so, x = _prefix_inputs(11, [4, 17, 1, 30], H=3, d=16)
+    o, _ = oracle.prefix_side_attention(x["q"], x["k"], x["v"], so)
+    for p in range(len(so) - 1):
+        a, b = so[p], so[p + 1]
+        t = lambda k: torch.from_numpy(np.ascontiguousarray(x[k][a:b].transpose(1, 0, 2)))[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(t("q"), t("k"), t("v"), is_causal=False)
+        np.testing.assert_allclose(o[a:b], ref[0].numpy().transpose(1, 0, 2), rtol=1e-12, atol=1e-13)
+
+
+def test_prefix_side_token_permutation_and_isolation():
+    so, x = _prefix_inputs(12, [6, 9])
+    o, _ = oracle.prefix_side_attention(x["q"], x["k"], x["v"], so)
+    perm = np.concatenate([np.random.default_rng(3).permutation(6), 6 + np.arange(9)])
+    xp = {k: v[perm] for k, v in x.items()}
+    op, _ = oracle.prefix_side_attention(xp["q"], xp["k"], xp["v"], so)
+    np.testing.assert_allclose(op, o[perm], rtol=1e-12, atol=1e-13)
+    # A prefix does not see another prefix's tokens: changing prefix 1 leaves prefix 0 alone.
+    x2 = {k: v.copy() for k, v in x.items()}
+    x2["k"][6:] += 5.0
+    x2["v"][6:] -= 3.0
+    o2, _ = oracle.prefix_side_attention(x2["q"], x2["k"], x2["v"], so)
+    np.testing.assert_array_equal(o2[:6], o[:6])
+    assert not np.allclose(o2[6:], o[6:])
+
+
 def test_requests_subset_and_empty_suffix():
     tab = RequestTable(np.array([3]), np.array([0, 0, -1]), np.array([2, 0, 3]))
     x = {k: as64(v) for k, v in host_tensors(tab, 1, 4, "fp32", 12).items()}

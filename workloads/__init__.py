@@ -40,6 +40,7 @@ __all__ = [
     "make_table",
     "split_launches",
     "random_table",
+    "prefix_side_table",
     "host_tensors",
     "device_tensors",
     "zipf_ranks",
@@ -196,6 +197,13 @@ def split_launches(table: RequestTable, n_launches: int) -> List[RequestTable]:
     R = table.R
     bounds = [(R * i) // n_launches for i in range(n_launches + 1)]
     return [table.subset(np.arange(bounds[i], bounds[i + 1])) for i in range(n_launches)]
+
+
+def prefix_side_table(table: "RequestTable") -> "RequestTable":
+    """The prefix-side batch of a workload: every prefix some request reads becomes one
+    request with no cached prefix whose own tokens are the prefix's tokens (lengths only)."""
+    used = table.referenced_prefixes()
+    return RequestTable(np.zeros(0, np.int64), np.full(len(used), -1, np.int32), table.prefix_len[used])
 
 
 def random_table(rng: np.random.Generator, P: int, R: int, max_prefix: int, max_suffix: int,
