@@ -361,61 +361,107 @@ def main():
     kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
     traffic = None if args.prefix_side else traffic_per_launch(args.workload, kernel_src)
 
-    # End to end through the public API with host buffers: per launch, H2D of the request
-    # tokens (q, k, v) from pinned memory, the forward, D2H of the output.  The prefix cache is
-    # resident (it is built once per cached prefix, off this path).
+    # End to end through the public API with host buffers: every launch's request tokens (q,
+    # k, v) go host -> device from pinned memory, the forward runs, the output comes back.  The
+    # prefix cache is resident (it is built once per cached prefix, off this path).  As a
+    # serving loop would, the launches are pipelined over two device buffer sets and three
+    # streams: the copy-in of launch i+1 and the copy-out of launch i-1 overlap the forward of
+    # launch i.  Each launch is split in two so that two buffer sets fit beside the cache.
     e2e = None
-    need_host = 4 * rows * spec.H * spec.d * 2
-    try:
-        import psutil
-        host_ok = psutil.virtual_memory().available > 1.5 * need_host
-    except Exception:
-        host_ok = True
-    if not args.no_e2e and not host_ok:
-        e2e = {"value": None, "unit": UNIT, "skipped": f"needs {need_host / 1e9:.0f} GB of pinned host memory"}
-    elif not args.no_e2e:
-        h = {k: torch.empty((rows, spec.H, spec.d), dtype=torch.bfloat16, pin_memory=True) for k in ("q", "k", "v", "o")}
-        for k, src in (("q", "q"), ("k", "k_suf"), ("v", "v_suf")):
-            h[k].copy_(suf[src])
+    row_b = spec.H * spec.d * 2
+    if not args.no_e2e:
+        for pl in plans:
+            pl.close()
+        suf = out = None
+        torch.cuda.empty_cache()
+        parts2 = split_launches(tab, 2 * n_launch)
+        rows2 = max(p.T_suf for p in parts2)
+        need_host = 4 * rows2 * row_b
+        try:
+            import psutil
+            host_ok = psutil.virtual_memory().available > 1.5 * need_host
+        except Exception:
+            host_ok = True
+        free_now, _ = torch.cuda.mem_get_info()
+        if not host_ok:
+            e2e = {"value": None, "unit": UNIT, "skipped": f"needs {need_host / 1e9:.0f} GB of pinned host memory"}
+        elif free_now < 0.9 * 2 * 4 * rows2 * row_b:
+            e2e = {"value": None, "unit": UNIT, "skipped": "two device buffer sets do not fit"}
+        else:
+            plans2 = [bat.Plan(p.req_prefix, p.suffix_offsets, p.prefix_offsets, spec.H, spec.d, bat.BAT_BF16)
+                      for p in parts2]
+            ws2 = torch.empty(max(max(pl.workspace_bytes for pl in plans2), 16), dtype=torch.uint8, device=dev)
+            h = {k: torch.empty((rows2, spec.H, spec.d), dtype=torch.bfloat16, pin_memory=True) for k in ("q", "k", "v", "o")}
+            sets = [{k: torch.empty((rows2, spec.H, spec.d), dtype=torch.bfloat16, device=dev) for k in ("q", "k", "v", "o")}
+                    for _ in range(2)]
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(seed + 2)
+            for k in ("q", "k", "v"):   # N(0,1) request tokens, drawn on the device, kept on the host
+                sets[0][k].normal_(generator=gen)
+                h[k].copy_(sets[0][k])
+            s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            for p, pl in zip(parts, plans):
-                T = p.T_suf
-                suf["q"][:T].copy_(h["q"][:T], non_blocking=True)
-                suf["k_suf"][:T].copy_(h["k"][:T], non_blocking=True)
-                suf["v_suf"][:T].copy_(h["v"][:T], non_blocking=True)
-                bat.bat_attention_forward(pl, suf["q"][:T], suf["k_suf"][:T], suf["v_suf"][:T], cache["k_cache"],
-                                          cache["v_cache"], out=out[:T], workspace=ws, stream=stream)
-                h["o"][:T].copy_(out[:T], non_blocking=True)
+            def e2e_step():
+                ev_run = [None, None]
+                ev_out = [None, None]
+                for i, (p, pl) in enumerate(zip(parts2, plans2)):
+                    T, b = p.T_suf, sets[i % 2]
+                    with torch.cuda.stream(s_in):
+                        # The buffer set is free once launch i-2 has read it and its output left.
+                        for ev in (ev_run[i % 2], ev_out[i % 2]):
+                            if ev is not None:
+                                s_in.wait_event(ev)
+                        b["q"][:T].copy_(h["q"][:T], non_blocking=True)
+                        b["k"][:T].copy_(h["k"][:T], non_blocking=True)
+                        b["v"][:T].copy_(h["v"][:T], non_blocking=True)
+                        ev_in = torch.cuda.Event()
+                        ev_in.record(s_in)
+                    s_run.wait_event(ev_in)
+                    bat.bat_attention_forward(pl, b["q"][:T], b["k"][:T], b["v"][:T], cache["k_cache"], cache["v_cache"],
+                                              out=b["o"][:T], workspace=ws2, stream=s_run)
+                    ev_run[i % 2] = torch.cuda.Event()
+                    ev_run[i % 2].record(s_run)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(ev_run[i % 2])
+                        h["o"][:T].copy_(b["o"][:T], non_blocking=True)
+                        ev_out[i % 2] = torch.cuda.Event()
+                        ev_out[i % 2].record(s_out)
+                return ev_out
 
-        e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
             e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        row_b = spec.H * spec.d * 2
-        e2e = {"value": step_flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": int(3 * tab.T_suf * row_b), "d2h_bytes_per_step": int(tab.T_suf * row_b),
-               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
-        del h
-        if bat.bat_get_device_status() != bat.BAT_OK:
-            raise RuntimeError(bat.last_error())
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s_in)
+            for _ in range(args.e2e_steps):
+                last = e2e_step()
+            for ev in last:
+                if ev is not None:
+                    s_out.wait_event(ev)
+            b_ev.record(s_out)
+            torch.cuda.synchronize()
+            e_ms = a.elapsed_time(b_ev)
+            if world > 1:
+                tt = torch.tensor([e_ms], device=dev)
+                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+                e_ms = float(tt.item())
+            e2e = {"value": step_flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+                   "h2d_bytes_per_step": int(3 * tab.T_suf * row_b), "d2h_bytes_per_step": int(tab.T_suf * row_b),
+                   "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
+                   "pipeline": f"{len(parts2)} launches over 2 buffer sets; copy-in, forward, copy-out on 3 streams"}
+            for pl in plans2:
+                pl.close()
+            del h, sets, ws2
+            if bat.bat_get_device_status() != bat.BAT_OK:
+                raise RuntimeError(bat.last_error())
+    else:
+        for pl in plans:
+            pl.close()
 
-    for pl in plans:
-        pl.close()
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        del suf, cache, out, ws
+        suf = cache = out = ws = None
         torch.cuda.empty_cache()
         base = cpu_baseline(args.workload, prefix_side=args.prefix_side)
 
