@@ -139,3 +139,29 @@ def test_group_items_are_contiguous_and_heaviest_group_first():
     # The hottest item (most requests) comes first.
     counts = np.bincount(tab.req_prefix, minlength=tab.P)
     assert groups[0] == np.argmax(counts)
+
+
+def test_prefix_side_plan_is_the_no_cache_plan():
+    """bat_plan_create_prefix_side: every prefix becomes a request with no cached prefix whose
+    own tokens are the prefix's, so its work list equals bat_plan_create's for that table."""
+    lens = [0, 1, 127, 128, 129, 300, 5, 1000]
+    tab = RequestTable(np.zeros(0, np.int64), np.full(len(lens), -1), np.array(lens))
+    with bat.Plan.prefix_side(tab.suffix_offsets, H=3, d=128, host_only=True) as p:
+        items, info = p.items(), p.info()
+    with plan_of(tab, H=3, d=128) as q:
+        ref = q.items()
+    assert info.P == 0 and info.R == len(lens) and info.T_cache == 0 and info.T_suf == sum(lens)
+    np.testing.assert_array_equal(items, ref)
+    assert (items["pre_len"] == 0).all()
+    check_plan(tab, H=3, d=128)
+
+
+def test_prefix_side_plan_argument_errors():
+    with pytest.raises(bat.BatError) as e:
+        bat.Plan.prefix_side(np.array([0, 5, 3]), H=2, d=64, host_only=True)   # not monotone
+    assert e.value.status == bat.BAT_ERR_INVALID_ARG
+    with pytest.raises(bat.BatError) as e:
+        bat.Plan.prefix_side(np.array([0, 5]), H=2, d=96, host_only=True)      # unsupported d
+    assert e.value.status == bat.BAT_ERR_UNSUPPORTED
+    with bat.Plan.prefix_side(np.array([0]), H=2, d=64, host_only=True) as p:  # no prefixes: empty plan
+        assert p.info().n_items == 0
