@@ -4,8 +4,10 @@
 // request's suffix rows attend, with no mask, over [cached prefix K/V ; own suffix K/V].
 // The prefix K/V is computed once and cached; every request that references it reuses it.
 //
-// One persistent CTA per SM walks the work list built by the host grouping pass.  A work
-// item holds one head and up to two 128-row query tiles (A, B) that read the same prefix.
+// One persistent CTA per SM takes work items from the list built by the host grouping pass,
+// in list order from a global counter (so the items of one prefix group run at the same time
+// on neighbouring SMs and share their K/V tiles through L2).  A work item holds one head and
+// up to two 128-row query tiles (A, B) that read the same prefix.
 // The CTA streams the item's key tiles through shared memory with TMA, once each, and both
 // query tiles consume every shared tile:
 //
@@ -15,9 +17,11 @@
 //   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V
 //                (d = 128: SS, P read from shared memory; d = 64: TS, P read from TMEM).  S of
 //                key tile j+1 is issued as soon as the softmax has read S of tile j, so it is
-//                computed while the softmax of tile j runs; PV of tile j follows its P.
+//                computed while the softmax of tile j runs; PV of tile j follows its P (at
+//                d = 64 in two 64-key halves, each as soon as its half of P is written).
 //   warp 11      idle (it completes the third warpgroup for the register split)
-//   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane)
+//   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane); the
+//                epilogue writes O / l through shared memory with bulk tensor stores
 //   warps 4..7   softmax + epilogue of tile B
 //
 // TMEM (512 columns): S_A, S_B (128 fp32 columns each), O_A, O_B (d columns each); at d = 64
