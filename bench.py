@@ -377,15 +377,26 @@ def main():
         parts2 = split_launches(tab, 2 * n_launch)
         rows2 = max(p.T_suf for p in parts2)
         need_host = 4 * rows2 * row_b
+        # Every rank on this node pins its own host buffers.
+        local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
         try:
             import psutil
-            host_ok = psutil.virtual_memory().available > 1.5 * need_host
+            host_ok = psutil.virtual_memory().available > 1.5 * need_host * local_world
         except Exception:
             host_ok = True
         free_now, _ = torch.cuda.mem_get_info()
+        fits = free_now >= 0.9 * 2 * 4 * rows2 * row_b
+        if world > 1:
+            # Every rank takes the same collective steps: agree on whether all ranks run it.
+            flag = torch.tensor([1 if (host_ok and fits) else 0], device=dev)
+            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+            host_ok, fits = bool(flag.item()) and host_ok, bool(flag.item()) and fits
+            if not (host_ok and fits):
+                host_ok = False
         if not host_ok:
-            e2e = {"value": None, "unit": UNIT, "skipped": f"needs {need_host / 1e9:.0f} GB of pinned host memory"}
-        elif free_now < 0.9 * 2 * 4 * rows2 * row_b:
+            e2e = {"value": None, "unit": UNIT,
+                   "skipped": f"needs {need_host * local_world / 1e9:.0f} GB of pinned host memory on this node"}
+        elif not fits:
             e2e = {"value": None, "unit": UNIT, "skipped": "two device buffer sets do not fit"}
         else:
             plans2 = [bat.Plan(p.req_prefix, p.suffix_offsets, p.prefix_offsets, spec.H, spec.d, bat.BAT_BF16)
