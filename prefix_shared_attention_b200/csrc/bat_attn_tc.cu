@@ -11,15 +11,16 @@
 // The CTA streams the item's key tiles through shared memory with TMA, once each, and both
 // query tiles consume every shared tile:
 //
-//   warp 8       TMA producer: Q tiles, then K/V tiles into a ring in the order the MMA
-//                issuers consume them: K0, K1, V0, K2, V1, ... (the K tile of key tile j+1
-//                ahead of the V tile of key tile j)
+//   warp 8       TMA producer: Q tiles, then the K tiles (d = 128) into a K ring, or (d = 64)
+//                the K and V tiles into one ring in the order the MMA issuers consume them:
+//                K0, K1, V0, K2, V1, ... (the K tile of key tile j+1 ahead of the V tile of j)
 //   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V
 //                (d = 128: SS, P read from shared memory; d = 64: TS, P read from TMEM).  S of
 //                key tile j+1 is issued as soon as the softmax has read S of tile j, so it is
 //                computed while the softmax of tile j runs; PV of tile j follows its P (at
 //                d = 64 in two 64-key halves, each as soon as its half of P is written).
-//   warp 11      idle (it completes the third warpgroup for the register split)
+//   warp 11      d = 128: TMA producer of the V tiles into a V ring; d = 64: idle (it
+//                completes the third warpgroup for the register split)
 //   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane); the
 //                epilogue writes O / l through shared memory with bulk tensor stores
 //   warps 4..7   softmax + epilogue of tile B
@@ -97,7 +98,6 @@ __device__ unsigned* g_phase;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
 constexpr int kItemQ = 4;                   // work items the producer may run ahead by
-constexpr int kItemConsumers = 10;          // 2 MMA warps + 8 softmax warps pop every item
 #ifdef BAT_FMA_EXP_PAIRS
 constexpr int kFmaExpPairsSet = BAT_FMA_EXP_PAIRS;   // build-time override, same for every d
 #else
@@ -351,7 +351,16 @@ struct Cfg {
   // One shared-memory tile per query tile: P (d = 128), and at the end of an item the staging
   // buffer of the output tile (both d).
   static constexpr int kPBufs = 2;
-  static constexpr int kStages = D == 128 ? 3 : 10;        // K/V ring depth (fills 227 KB)
+  // K/V ring depth (fills 227 KB).  d = 128: three tiles, split into a K ring of two and a V
+  // ring of one, each with its own producer warp, so a K tile is never queued behind a V tile
+  // (measured 1-2% faster than one shared ring of three).  d = 64: one ring of ten, filled in
+  // consumption order by one producer (every split of it measured slower).
+  static constexpr bool kTwoRings = D == 128;
+  static constexpr int kStages = D == 128 ? 3 : 10;
+  static constexpr int kStagesK = kTwoRings ? 2 : kStages;
+  static constexpr int kStagesV = kStages - kStagesK;
+  // Warps that pop every work item: 8 softmax, 2 MMA issuers and, with two rings, the V producer.
+  static constexpr int kItemConsumers = kTwoRings ? 11 : 10;
   // d = 64: PV is issued in two halves of 64 keys, each as soon as the softmax has written that
   // half of P, so the next tile's P can overwrite the first half early (measured faster at
   // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
@@ -476,9 +485,9 @@ template <int D>
 struct Smem {
   uint8_t* q;        // [2][kTileBytes]
   uint8_t* p;        // [kPBufs][kTileBytes]: P of tiles A, B (d = 128) / output staging
-  uint8_t* kv;       // [kStages][kTileBytes]
-  uint64_t* kv_full;
-  uint64_t* kv_empty;
+  uint8_t* kv;       // [kStages][kTileBytes]: the K ring (or the shared ring), then the V ring
+  uint64_t* kv_full;   // [kStages]
+  uint64_t* kv_empty;  // [kStages]
   uint64_t* q_full;   // [2]
   uint64_t* q_empty;  // [2]
   uint64_t* s_full;   // [2]
@@ -510,6 +519,53 @@ __device__ __forceinline__ int pop_item(const Smem<D>& sm, uint32_t& k, const Ct
 
 // ------------------------------------------------------------------------------------
 // Roles
+
+// The rings of K/V tiles: the K ring and the V ring (two producers), or one ring that holds
+// both in consumption order (one producer).  Slot of ring sequence number r: first(R) + r % depth(R).
+enum Ring { kRingK = 0, kRingV = 1, kRingKV = 2 };
+template <int D, int R>
+struct RingGeom {
+  static constexpr uint32_t kDepth = R == kRingK ? Cfg<D>::kStagesK : R == kRingV ? Cfg<D>::kStagesV : Cfg<D>::kStages;
+  static constexpr uint32_t kFirst = R == kRingV ? Cfg<D>::kStagesK : 0;
+};
+
+// Loads one item's tiles of ring R, in the order the MMA issuers consume them; `ring` counts
+// the loads this warp has issued into R.  Returns false on abort.
+template <int D, int R>
+__device__ __forceinline__ bool load_ring(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, const WorkItem& w,
+                                          const Stream& st, uint32_t& ring) {
+  using C = Cfg<D>;
+  using G = RingGeom<D, R>;
+  const int lane = threadIdx.x & 31;
+  const int npos = R == kRingKV ? 2 * st.n : st.n;
+  for (int pos = 0; pos < npos; ++pos) {
+    int j = pos, mask, row0;
+    bool is_v = R == kRingV, from_cache;
+    if (R == kRingKV) st.slot(pos, j, is_v);
+    st.tile(w, j, mask, from_cache, row0);
+    const uint32_t s = G::kFirst + ring % G::kDepth, ph = (ring / G::kDepth) & 1;
+    if (!wait_bar(sm.kv_empty + s, ph ^ 1, ctl)) return false;
+    if (lane == 0) {
+      const CUtensorMap* m = from_cache ? (is_v ? &p.tm_vc : &p.tm_kc) : (is_v ? &p.tm_vs : &p.tm_ks);
+      mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn)
+        tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, w.head * D + pn * 64, row0,
+                    sm.kv_full + s);
+    }
+    __syncwarp();
+    ++ring;
+  }
+  return true;
+}
+
+// After an abort: waits (bounded) for the last loads issued into ring R to land.
+template <int D, int R>
+__device__ __forceinline__ void drain_ring(const Smem<D>& sm, uint32_t ring) {
+  using G = RingGeom<D, R>;
+  const uint32_t n = ring < G::kDepth ? ring : G::kDepth;
+  for (uint32_t i = ring - n; i < ring; ++i) drain_bar(sm.kv_full + G::kFirst + i % G::kDepth, (i / G::kDepth) & 1);
+}
 
 template <int D>
 __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl) {
@@ -553,35 +609,33 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
       ++qcnt[x];
     }
     const Stream st(w);
-    for (int pos = 0; ok && pos < 2 * st.n; ++pos) {
-      int j, mask, row0;
-      bool is_v, from_cache;
-      st.slot(pos, j, is_v);
-      st.tile(w, j, mask, from_cache, row0);
-      const uint32_t s = ring % C::kStages, ph = (ring / C::kStages) & 1;
-      ok = wait_bar(sm.kv_empty + s, ph ^ 1, ctl);
-      if (!ok) break;
-      if (pos < 2 || pos == 2 * st.n - 1) BAT_TRACE_EV(0, tn, 3 + (pos == 2 * st.n - 1 ? 2 : pos), 0, kq);
-      if (lane == 0) {
-        const CUtensorMap* m = from_cache ? (is_v ? &p.tm_vc : &p.tm_kc) : (is_v ? &p.tm_vs : &p.tm_ks);
-        mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, w.head * D + pn * 64, row0,
-                      sm.kv_full + s);
-      }
-      __syncwarp();
-      ++ring;
-    }
+    ok = load_ring<D, C::kTwoRings ? kRingK : kRingKV>(p, sm, ctl, w, st, ring);
   }
   BAT_PHASE_FLUSH();
   if (!ok && lane == 0) {
     // Let every copy this warp issued land before the CTA releases its shared memory.
-    const uint32_t n = ring < (uint32_t)C::kStages ? ring : (uint32_t)C::kStages;
-    for (uint32_t i = ring - n; i < ring; ++i) drain_bar(sm.kv_full + i % C::kStages, (i / C::kStages) & 1);
+    drain_ring<D, C::kTwoRings ? kRingK : kRingKV>(sm, ring);
     for (int x = 0; x < 2; ++x)
       if (qcnt[x]) drain_bar(sm.q_full + x, (qcnt[x] - 1) & 1);
   }
+  __syncwarp();
+}
+
+// V producer (warp 11, d = 128): the value tiles of every item, in key-tile order, into the
+// V ring.  It pops the same work items as every other role.
+template <int D>
+__device__ void vproducer_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ring = 0, kq = 0;
+  bool ok = true;
+  while (ok) {
+    const int it = pop_item<D>(sm, kq, ctl, ok);
+    if (it < 0) break;
+    const WorkItem w = p.items[it];
+    const Stream st(w);
+    ok = load_ring<D, kRingV>(p, sm, ctl, w, st, ring);
+  }
+  if (!ok && lane == 0) drain_ring<D, kRingV>(sm, ring);
   __syncwarp();
 }
 
@@ -592,16 +646,18 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
 // two arrivals, one per issuer: a commit after its MMAs read the slot, or, for a tile this
 // query tile does not read, a plain arrive once the tile has landed.
 //
-// Each issuer walks the ring positions in order (K0, K1, V0, K2, V1, ...): S of key tile j+1
-// waits only for the softmax to have read S of tile j (S has its own TMEM columns), so it is
-// computed while that softmax runs; PV of tile j waits for its P.  Because every wait is on
-// the issuer's current ring position or on its own softmax, which only needs earlier
-// positions, no ring depth can deadlock.
+// Each issuer takes the tiles in one order (K0, K1, V0, K2, V1, ...), which is also the order
+// of the shared ring and the order of each of the two rings: S of key tile j+1 waits only for
+// the softmax to have read S of tile j (S has its own TMEM columns), so it is computed while
+// that softmax runs; PV of tile j waits for its P.  Every wait is on the issuer's next tile or
+// on its own softmax, which only needs earlier tiles, and every slot is freed by tiles earlier
+// in that order, so no ring depth can deadlock (with two rings the producers also share only
+// the work-item queue, which they both pop in order).
 template <int D>
 __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, uint32_t tmem, int X) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t ring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
+  uint32_t ring = 0, vring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
   bool ok = true;
   int tn = 0;
   (void)tn;
@@ -620,8 +676,15 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
     if (it < 0) break;
     const WorkItem w = p.items[it];
     const Stream st(w);
-    const uint32_t ring0 = ring;
-    ring += 2u * st.n;
+    // Sequence numbers of the item's first K and V tiles in their rings (one shared ring at
+    // d = 64, where the item's position pos is its sequence number).
+    const uint32_t kr0 = ring, vr0 = vring;
+    if constexpr (C::kTwoRings) {
+      ring += (uint32_t)st.n;
+      vring += (uint32_t)st.n;
+    } else {
+      ring += 2u * st.n;
+    }
     const bool mine = X < w.n_q;
     int s_left = mine ? st.count(X) : 0;
     bool first_s = true, first_pv = true;
@@ -630,9 +693,18 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
       bool is_v, from_cache;
       st.slot(pos, j, is_v);
       st.tile(w, j, mask, from_cache, row0);
-      const uint32_t r = ring0 + pos, s = r % C::kStages;
+      uint32_t s, ph;
+      if constexpr (C::kTwoRings) {
+        const uint32_t r = (is_v ? vr0 : kr0) + j;
+        s = is_v ? RingGeom<D, kRingV>::kFirst + r % C::kStagesV : r % C::kStagesK;
+        ph = (r / (is_v ? C::kStagesV : C::kStagesK)) & 1;
+      } else {
+        const uint32_t r = kr0 + pos;
+        s = r % C::kStages;
+        ph = (r / C::kStages) & 1;
+      }
       if (pos == 0) BAT_TRACE_EV(1 + X, tn, 6, X, s_issued);
-      ok = wait_bar(sm.kv_full + s, (r / C::kStages) & 1, ctl);
+      ok = wait_bar(sm.kv_full + s, ph, ctl);
       if (!ok) break;
       if (!mine || !((mask >> X) & 1)) {
         // A tile this query tile does not read: release the slot once it has landed.
@@ -993,7 +1065,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     mbar_init(sm.drain + 1, 1);
     for (int i = 0; i < kItemQ; ++i) {
       mbar_init(sm.itq_full + i, 1);
-      mbar_init(sm.itq_empty + i, kItemConsumers);
+      mbar_init(sm.itq_empty + i, C::kItemConsumers);
     }
     *sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1018,13 +1090,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   const uint32_t tmem = *sm.tmem_slot;
   const Ctl ctl{sm.abort_flag, p.status, p.wait_ns};
 
-  // Register split: the control warpgroup (producer, MMA issuer, two idle warps) gives up
+  // Register split: the control warpgroup (producers, MMA issuers, idle warp) gives up
   // registers to the two softmax warpgroups.  384 threads x 168 at launch = 64512 =
   // 128 x 104 + 256 x 200.
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
     if (warp == 8) producer_role<D>(p, sm, ctl);
     else if (warp == 9 || warp == 10) mma_role<D>(p, sm, ctl, tmem, warp - 9);
+    else if constexpr (C::kTwoRings) vproducer_role<D>(p, sm, ctl);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
     softmax_role<D>(p, sm, ctl, tmem, warp >> 2);
