@@ -62,6 +62,72 @@ def traffic_per_launch(workload, kernel_src):
     return rec.get("dram_bytes_per_launch") if rec.get("kernel_sha256_16") == h else None
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event-reason samples read through NVML (read only) every `period_s`
+    while the timed region runs, plus one at its end, so a timed region shorter than a
+    polling interval still has a record.  The device is found by its UUID, so the right GPU
+    is read whatever CUDA_VISIBLE_DEVICES maps.  `nvml` is the binding module (injectable)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, uuid, nvml=None, period_s=0.002):
+        self.uuid, self.nvml, self.period = uuid, nvml, period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self.thread = None
+
+    def _sample(self):
+        n = self.nvml
+        self.samples.append((n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM),
+                             n.nvmlDeviceGetMaxClockInfo(self.h, n.NVML_CLOCK_SM),
+                             n.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+
+    def start(self):
+        if self.nvml is None:
+            import pynvml
+            self.nvml = pynvml
+        self.nvml.nvmlInit()
+        u = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+        self.h = self.nvml.nvmlDeviceGetHandleByUUID(u)
+        self._sample()   # the binding works: fail here, before the timed region, if it does not
+
+        def run():
+            while not self._stop.wait(self.period):
+                self._sample()
+        self.samples.clear()
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        self._stop.set()
+        self.thread.join(timeout=2)
+        self._sample()
+        try:
+            self.nvml.nvmlShutdown()
+        except Exception:
+            pass
+        sm = [c for c, _, _ in self.samples]
+        reasons = sorted({name for _, _, r in self.samples for name, attr in self.REASONS
+                          if r & getattr(self.nvml, attr)})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(m for _, m, _ in self.samples),
+                "reasons": reasons, "samples": len(sm), "source": "nvml"}
+
+
+def clock_sampler(dev_index):
+    """NVML sampler of this process's GPU, else the nvidia-smi one."""
+    import torch
+    try:
+        s = NvmlClockSampler(str(torch.cuda.get_device_properties(dev_index).uuid))
+        s.start()
+        s.stop()
+        return NvmlClockSampler(s.uuid, s.nvml)
+    except Exception:
+        return ClockSampler(dev_index)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -112,7 +178,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 def fits_launches(tab, spec, free_bytes, elt):
@@ -321,7 +387,7 @@ def main():
 
     ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in parts] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
+    clocks = clock_sampler(local_rank)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
