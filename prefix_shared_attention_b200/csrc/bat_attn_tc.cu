@@ -45,6 +45,12 @@
 namespace bat {
 namespace {
 
+// A compile-time bool as a type (selects one of the two compiled copies of the softmax tile).
+template <bool B>
+struct BoolC {
+  static constexpr bool value = B;
+};
+
 __device__ uint32_t g_status_word;
 
 // Compile-time event trace of CTA 0 (off unless built with -DBAT_TRACE): per role, a list of
@@ -374,6 +380,12 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t o_col(int x) { return 256u + (uint32_t)D * x; }
   __host__ __device__ static constexpr uint32_t p_col(int x) { return 384u + 64u * x; }   // d = 64 only
   static constexpr uint32_t kIdescS = make_idesc(128, 128, false);
+  static constexpr uint32_t kIdescSHalf = make_idesc(128, 64, false);   // key tiles of <= 64 valid keys
+  // d = 64: a key tile with at most 64 valid keys (a short prefix, the ragged end of a stream)
+  // gets S at N = 64, PV over its first 64 keys and no exponentials or P stores for the masked
+  // half (measured +4 % on item-as-prefix, whose prefixes are 32 keys long).  At d = 128 the
+  // same skip made the full-tile softmax slower, so it is off there.
+  static constexpr bool kHalfSkip = D == 64;
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
   static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 4 + 4 * 2 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kPBufs + kStages) * kTileBytes + kBarBytes;
@@ -420,6 +432,16 @@ struct Stream {
     }
     mask = 1 << x;
     row0 = (x ? w.sB_row0 : w.sA_row0) + idx * kTileN;
+  }
+  // Valid keys in global tile j (the rest of the tile belongs to other rows: masked).
+  __device__ __forceinline__ int tile_valid(const WorkItem& w, int j) const {
+    if (j < npre) return min(kTileN, w.pre_len - j * kTileN);
+    const int k = j - npre;
+    if (shared) return min(kTileN, w.sA_len - k * kTileN);
+    const int mm = nsA < nsB ? nsA : nsB;
+    const int x = k < 2 * mm ? (k & 1) : (nsA > nsB ? 0 : 1);
+    const int idx = k < 2 * mm ? (k >> 1) : mm + (k - 2 * mm);
+    return min(kTileN, (x ? w.sB_len : w.sA_len) - idx * kTileN);
   }
   // Ring position pos (0 .. 2n-1) of the item's K/V loads: K0, K1, V0, K2, V1, ..., K(n-1),
   // V(n-2), V(n-1).  This is the order in which each MMA issuer uses them (S of key tile j+1,
@@ -725,10 +747,13 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         if (!ok) break;
         tc_fence_after();
         const uint64_t kd = kdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
+        // A key tile with at most 64 valid keys: S over its first 64 keys only (the softmax
+        // masks the other columns).
+        const uint32_t idS = (C::kHalfSkip && st.tile_valid(w, j) <= 64) ? C::kIdescSHalf : C::kIdescS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4);
-          mma_ss_w(s_t, qdesc + off, kd + off, C::kIdescS, kk > 0 ? 1u : 0u);
+          mma_ss_w(s_t, qdesc + off, kd + off, idS, kk > 0 ? 1u : 0u);
         }
         tc_commit_w(sm.s_full + X);
         if (s_left == 1) tc_commit_w(sm.q_empty + X);
@@ -742,6 +767,8 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         // the whole tile).  16 keys per instruction = two 8-row swizzle groups of V (2 KiB); LBO
         // steps between V's 64-column panels.
         const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
+        // P over keys 64 .. 127 of a tile with at most 64 valid keys is zero: skip those steps.
+        const int kk_end = (C::kHalfSkip && st.tile_valid(w, j) <= 64) ? 4 : 8;
 #pragma unroll
         for (int h = 2 - C::kPVHalves; h < 2; ++h) {
           BAT_TRACE_EV(1 + X, tn, 3, X, p_seen);
@@ -750,6 +777,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
           tc_fence_after();
 #pragma unroll
           for (int kk = C::kPVHalves == 2 ? 4 * h : 0; kk < 4 * h + 4; ++kk) {
+            if (kk >= kk_end) break;
             const uint32_t acc = (first_pv && kk == 0) ? 0u : 1u;
             const uint64_t vk = vd + (uint64_t)(kk * 2048 / 16);
             if constexpr (C::kPSmem) {
@@ -833,98 +861,120 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
       // S is in registers: the issuer may compute the next S into these columns.
       tc_fence_before();
       mbar_arrive(sm.s_free + X);
-      if (valid < kTileN) {
+      // The tile body; with kHalfSkip compiled twice: for full tiles and for tiles with at most
+      // 64 valid keys.
+      auto tile_body = [&](auto half_c) {
+        constexpr bool HALF = decltype(half_c)::value;
+        if (valid < kTileN) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = c < valid ? s[c] : -INFINITY;
-      }
-      // Row maximum: eight independent 3-input-max chains (short dependency depth).
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        mx[k] = s[16 * k];
-#pragma unroll
-        for (int i = 1; i < 15; i += 2) mx[k] = max3f(mx[k], s[16 * k + i], s[16 * k + i + 1]);
-        mx[k] = fmaxf(mx[k], s[16 * k + 15]);
-      }
-      const float tile_m = fmaxf(max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), mx[6]), mx[7]) * sl2;
-      float m_new = m;
-      if (t == 0) m_new = tile_m;
-      else if (tile_m > m + kRescaleThreshold) m_new = tile_m;
-      const bool resc = t > 0 && m_new != m;
-      if (__any_sync(0xffffffffu, resc)) {
-        // O holds the previous tiles' sum: wait for the last PV, then rescale in place.
-        ok = wait_bar(sm.pv_done + 2 * X + 1, (pv_base + t - 1) & 1, ctl);
-        if (!ok) break;
-        tc_fence_after();
-        const float alpha = resc ? ex2(m - m_new) : 1.f;
-        l *= alpha;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+          for (int c = 0; c < 128; ++c) s[c] = c < valid ? s[c] : -INFINITY;
         }
-        tmem_st_wait();
-      }
-      m = m_new;
-      BAT_TRACE_EV(3 + X, tn, 8, X, s_seen);
-      const float nm = -m;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
-      // stored (TMEM or shared memory, asynchronously) while the next half's exponentials run.
-      // Of every eight columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the
-      // MUFU.
+        // Row maximum: eight independent 3-input-max chains (short dependency depth); four over
+        // the first 64 columns for a tile with at most 64 valid keys.
+        float mx[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int c = 64 * h; c < 64 * h + 64; c += 8) {
-#pragma unroll
-          for (int k = 0; k < 8; k += 2) ffma2(s[c + k], s[c + k + 1], s[c + k], s[c + k + 1], sl2, nm);
-#pragma unroll
-          for (int k = 0; k < 8 - 2 * C::kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
-#pragma unroll
-          for (int k = 8 - 2 * C::kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
-          fadd2(a0, a1, s[c], s[c + 1]);
-          fadd2(a2, a3, s[c + 2], s[c + 3]);
-          fadd2(a0, a1, s[c + 4], s[c + 5]);
-          fadd2(a2, a3, s[c + 6], s[c + 7]);
-        }
-        if (t > 0 && (C::kPVHalves == 2 || h == 0)) {
-          // This half of the previous P (with one PV part: all of it) must have been consumed
-          // before it is overwritten.
-          BAT_TRACE_EV(3 + X, tn, 12, X, s_seen);
-          ok = wait_bar(sm.pv_done + 2 * X + (C::kPVHalves == 2 ? h : 1), (pv_base + t - 1) & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          BAT_TRACE_EV(3 + X, tn, 11, X, s_seen);
-        }
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]);
-        if constexpr (C::kPSmem) {
-          // Keys 64h .. 64h+63 are panel h of the P tile.
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
-            st_shared_v4(p_row + h * C::kPanelBytes + ((cc ^ p_sw) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
-                         pk[4 * cc + 3]);
-        } else {
-          tmem_st32(tP + 32 * h, pk);
-        }
-        if (C::kPVHalves == 2 || h == 1) {
-          if constexpr (C::kPSmem) {
-            // Make the generic-proxy stores visible to the tensor core (async proxy).
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          } else {
-            tmem_st_wait();
-            tc_fence_before();
+        for (int k = 0; k < 8; ++k) {
+          if (HALF && k >= 4) {
+            mx[k] = -INFINITY;
+            continue;
           }
-          mbar_arrive(sm.p_full + 2 * X + h);
+          mx[k] = s[16 * k];
+#pragma unroll
+          for (int i = 1; i < 15; i += 2) mx[k] = max3f(mx[k], s[16 * k + i], s[16 * k + i + 1]);
+          mx[k] = fmaxf(mx[k], s[16 * k + 15]);
         }
+        const float tile_m = fmaxf(max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), mx[6]), mx[7]) * sl2;
+        float m_new = m;
+        if (t == 0) m_new = tile_m;
+        else if (tile_m > m + kRescaleThreshold) m_new = tile_m;
+        const bool resc = t > 0 && m_new != m;
+        if (__any_sync(0xffffffffu, resc)) {
+          // O holds the previous tiles' sum: wait for the last PV, then rescale in place.
+          ok = wait_bar(sm.pv_done + 2 * X + 1, (pv_base + t - 1) & 1, ctl);
+          if (!ok) return;
+          tc_fence_after();
+          const float alpha = resc ? ex2(m - m_new) : 1.f;
+          l *= alpha;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+          tmem_st_wait();
+        }
+        m = m_new;
+        BAT_TRACE_EV(3 + X, tn, 8, X, s_seen);
+        const float nm = -m;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
+        // stored (TMEM or shared memory, asynchronously) while the next half's exponentials run.
+        // Of every eight columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the
+        // MUFU.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // A tile with at most 64 valid keys: keys 64 .. 127 carry no weight and PV skips them,
+          // so their exponentials and P stores are skipped (the barrier hand-offs stay).
+          const bool skip = HALF && h == 1;
+#pragma unroll
+          for (int c = 64 * h; c < 64 * h + 64; c += 8) {
+            if (skip) break;
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) ffma2(s[c + k], s[c + k + 1], s[c + k], s[c + k + 1], sl2, nm);
+#pragma unroll
+            for (int k = 0; k < 8 - 2 * C::kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
+#pragma unroll
+            for (int k = 8 - 2 * C::kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
+            fadd2(a0, a1, s[c], s[c + 1]);
+            fadd2(a2, a3, s[c + 2], s[c + 3]);
+            fadd2(a0, a1, s[c + 4], s[c + 5]);
+            fadd2(a2, a3, s[c + 6], s[c + 7]);
+          }
+          if (t > 0 && (C::kPVHalves == 2 || h == 0)) {
+            // This half of the previous P (with one PV part: all of it) must have been consumed
+            // before it is overwritten.
+            BAT_TRACE_EV(3 + X, tn, 12, X, s_seen);
+            ok = wait_bar(sm.pv_done + 2 * X + (C::kPVHalves == 2 ? h : 1), (pv_base + t - 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            BAT_TRACE_EV(3 + X, tn, 11, X, s_seen);
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]);
+          if (skip) {
+          } else if constexpr (C::kPSmem) {
+            // Keys 64h .. 64h+63 are panel h of the P tile.
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+              st_shared_v4(p_row + h * C::kPanelBytes + ((cc ^ p_sw) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
+                           pk[4 * cc + 3]);
+          } else {
+            tmem_st32(tP + 32 * h, pk);
+          }
+          if (C::kPVHalves == 2 || h == 1) {
+            if constexpr (C::kPSmem) {
+              // Make the generic-proxy stores visible to the tensor core (async proxy).
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            } else {
+              tmem_st_wait();
+              tc_fence_before();
+            }
+            mbar_arrive(sm.p_full + 2 * X + h);
+          }
+        }
+        if (!ok) return;
+        l += (a0 + a1) + (a2 + a3);
+      };
+      if constexpr (C::kHalfSkip) {
+        if (valid <= 64) tile_body(BoolC<true>{});
+        else tile_body(BoolC<false>{});
+      } else {
+        tile_body(BoolC<false>{});
       }
       if (!ok) break;
-      l += (a0 + a1) + (a2 + a3);
       BAT_TRACE_EV(3 + X, tn, 2, X, s_seen);
     }
     if (!ok) break;
