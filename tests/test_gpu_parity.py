@@ -111,6 +111,21 @@ def test_edge_lengths(d):
 
 
 @pytest.mark.parametrize("d", [64, 128])
+def test_short_key_tiles(d):
+    # Key tiles with at most 32 or 64 valid keys (short prefixes and ragged stream ends), for
+    # which the d = 64 kernel computes only the first 64 key columns; the 63-key prefix
+    # carries the row maximum, so a rescale happens on a short tile.
+    pre = np.array([1, 31, 32, 33, 63, 64, 65, 96])
+    tab = RequestTable(pre, np.array([0, 1, 2, 3, 4, 5, 6, 7, 5, 4], np.int32),
+                       np.array([64, 160, 192, 129, 191, 33, 64, 200, 130, 63]))
+
+    def mutate(x):
+        x["k_cache"][int(pre[:4].sum()):int(pre[:5].sum())] *= 8.0
+
+    full_parity(tab, 2, d, "bf16", 21, mutate=mutate)
+
+
+@pytest.mark.parametrize("d", [64, 128])
 def test_explicit_scale(d):
     rng = np.random.default_rng(77)
     tab = random_table(rng, P=2, R=4, max_prefix=300, max_suffix=300)
