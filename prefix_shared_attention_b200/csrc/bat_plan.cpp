@@ -203,19 +203,47 @@ int build_plan(const int32_t* req_prefix, const int64_t* suffix_offsets,
   // Order: heaviest group first; within a group, every head in turn, items heaviest first.
   std::stable_sort(groups.begin(), groups.end(),
                    [](const Group& a, const Group& b) { return a.cost > b.cost; });
-  std::vector<WorkItem> items;
-  std::vector<MergeJob> merges;
-  int64_t n_slots = 0;
-  for (auto& g : groups) {
+  // Chunk counts per group item (the same for every head), and the exact output sizes.
+  std::vector<std::vector<int32_t>> nchs(groups.size());
+  int64_t n_items_total = 0, n_merges_total = 0;
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    auto& g = groups[gi];
     std::stable_sort(g.items.begin(), g.items.end(),
                      [](const WorkItem& a, const WorkItem& b) { return a.cost > b.cost; });
+    nchs[gi].resize(g.items.size());
+    for (size_t i = 0; i < g.items.size(); ++i) {
+      const int32_t nch = chunks_for(g.items[i]);
+      nchs[gi][i] = nch;
+      n_items_total += (int64_t)nch * H;
+      if (nch > 1) n_merges_total += (int64_t)g.items[i].n_q * H;
+    }
+  }
+  // The work list is written straight into the result's buffers.
+  if (n_items_total > 0) {
+    out->items = (WorkItem*)malloc((size_t)n_items_total * sizeof(WorkItem));
+    if (!out->items) return fail(err, err_len, "out of host memory for %lld work items", (long long)n_items_total);
+  }
+  if (n_merges_total > 0) {
+    out->merges = (MergeJob*)malloc((size_t)n_merges_total * sizeof(MergeJob));
+    if (!out->merges) {
+      free_plan_result(out);
+      return fail(err, err_len, "out of host memory for %lld merge jobs", (long long)n_merges_total);
+    }
+  }
+  WorkItem* items = out->items;
+  MergeJob* merges = out->merges;
+  int64_t ni = 0, nm = 0;
+  int64_t n_slots = 0;
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    const auto& g = groups[gi];
     for (int32_t h = 0; h < H; ++h) {
-      for (const WorkItem& w0 : g.items) {
-        const int32_t nch = chunks_for(w0);
+      for (size_t ii = 0; ii < g.items.size(); ++ii) {
+        const WorkItem& w0 = g.items[ii];
+        const int32_t nch = nchs[gi][ii];
         if (nch <= 1) {
-          WorkItem w = w0;
+          WorkItem& w = items[ni++];
+          w = w0;
           w.head = h;
-          items.push_back(w);
           continue;
         }
         const int64_t npre = cdiv(w0.pre_len, kTileN);
@@ -237,7 +265,7 @@ int build_plan(const int32_t* req_prefix, const int64_t* suffix_offsets,
           w.sB_row0 = w.sA_row0;
           w.sB_len = w.sA_len;
           w.cost = (int32_t)item_cost(w);
-          items.push_back(w);
+          items[ni++] = w;
         }
         n_slots += (int64_t)nch * w0.n_q;
         for (int32_t x = 0; x < w0.n_q; ++x) {
@@ -249,31 +277,24 @@ int build_plan(const int32_t* req_prefix, const int64_t* suffix_offsets,
           m.slot0 = (int32_t)(slot0 + x);
           m.n_chunks = nch;
           m.slot_stride = w0.n_q;
-          merges.push_back(m);
+          merges[nm++] = m;
         }
       }
     }
   }
-  if (n_slots > std::numeric_limits<int32_t>::max() / 2)
+  if (n_slots > std::numeric_limits<int32_t>::max() / 2) {
+    free_plan_result(out);
     return fail(err, err_len, "too many split slots (%lld)", n_slots);
-
-  out->n_items = (int64_t)items.size();
-  out->n_merges = (int64_t)merges.size();
+  }
+  if (ni != n_items_total || nm != n_merges_total) {
+    free_plan_result(out);
+    return fail(err, err_len, "internal: %lld work items and %lld merge jobs written, not the sizes counted",
+                (long long)ni, (long long)nm);
+  }
+  out->n_items = ni;
+  out->n_merges = nm;
   out->n_slots = n_slots;
   out->total_cost = total_cost;
-  if (!items.empty()) {
-    out->items = (WorkItem*)malloc(items.size() * sizeof(WorkItem));
-    if (!out->items) return fail(err, err_len, "out of host memory for %lld work items", (long long)items.size());
-    memcpy(out->items, items.data(), items.size() * sizeof(WorkItem));
-  }
-  if (!merges.empty()) {
-    out->merges = (MergeJob*)malloc(merges.size() * sizeof(MergeJob));
-    if (!out->merges) {
-      free_plan_result(out);
-      return fail(err, err_len, "out of host memory for %lld merge jobs", (long long)merges.size());
-    }
-    memcpy(out->merges, merges.data(), merges.size() * sizeof(MergeJob));
-  }
   return 0;
 }
 
