@@ -117,3 +117,20 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cpp", ".h")):
                 text = open(os.path.join(root, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_plain_c_consumer(tmp_path):
+    """The ABI from plain C: tests/c_consumer/plan_consumer.c, compiled with gcc against
+    include/bat.h and linked to libbat.so, builds host-only plans and checks error codes."""
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc is not installed")
+    lib_dir = os.path.dirname(bat.LIB_PATH)
+    exe = str(tmp_path / "plan_consumer")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_consumer", "plan_consumer.c"), "-L", lib_dir, "-lbat",
+                    f"-Wl,-rpath,{lib_dir}", "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "c consumer: ok" in r.stdout
