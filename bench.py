@@ -37,12 +37,23 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 2**20
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def load_peaks(path=None):
+    """The roofline denominators: each of hbm_gbs, bf16_tflops and bf16_tflops_sustained from
+    MEASURED_PEAKS.json when it holds a positive number for it, else the recorded fallback.
+    Returns (peaks, kinds) with kinds[key] in {"measured", "fallback"}."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = {}
     if os.path.exists(p):
-        d = json.load(open(p))
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        try:
+            d = json.load(open(p))
+        except (OSError, ValueError):
+            d = {}
+    peaks, kinds = {}, {}
+    for k, fb in FALLBACK_PEAKS.items():
+        v = d.get(k)
+        ok = isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0
+        peaks[k], kinds[k] = (float(v), "measured") if ok else (fb, "fallback")
+    return peaks, kinds
 
 
 def workload_flops_bytes(tab, H, d, elt):
@@ -414,7 +425,7 @@ def main():
     ms_per_step = elapsed_ms / args.steps
     value = step_flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
     req_s = tab.R * world * args.steps / (elapsed_ms * 1e-3)
-    peaks, peak_kind = load_peaks()
+    peaks, peak_kinds = load_peaks()
     achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
     # Which roof binds: algorithmic FLOP per byte against the ridge of the measured peaks.
     ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
@@ -556,8 +567,9 @@ def main():
             "plan_ms": plan_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_kind} " + ("bf16_tflops_sustained (timed region %.1f s under the power cap)"
-                                                           % (elapsed_ms / 1e3) if sustained else "bf16_tflops (burst)"),
+                         "peak_source": (f"{peak_kinds['bf16_tflops_sustained']} bf16_tflops_sustained (timed region "
+                                         f"{elapsed_ms / 1e3:.1f} s under the power cap)" if sustained
+                                         else f"{peak_kinds['bf16_tflops']} bf16_tflops (burst)"),
                          "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_of_spec": achieved / 2250.0,
@@ -572,7 +584,7 @@ def main():
             gbs = step_bytes / (sum(kernel_ms) * 1e-3) / 1e9
             line["roofline"].update({"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                      "frac": gbs / float(peaks["hbm_gbs"]),
-                                     "peak_source": f"{peak_kind} hbm_gbs", "tensor_tflops": achieved})
+                                     "peak_source": f"{peak_kinds['hbm_gbs']} hbm_gbs", "tensor_tflops": achieved})
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

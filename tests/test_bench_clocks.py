@@ -83,3 +83,17 @@ def test_nvidia_smi_sampler_without_the_tool():
     s.proc = None
     rec = s.stop()
     assert rec["sm_mhz"] is None and rec["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_peaks_fill_missing_keys_from_the_fallback(tmp_path):
+    bench = load_bench()
+    p = tmp_path / "peaks.json"
+    p.write_text('{"hbm_gbs": 6400.0, "bf16_tflops": "n/a", "sm_max_mhz": 1965}')
+    peaks, kinds = bench.load_peaks(str(p))
+    assert peaks["hbm_gbs"] == 6400.0 and kinds["hbm_gbs"] == "measured"
+    assert peaks["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"] and kinds["bf16_tflops"] == "fallback"
+    assert kinds["bf16_tflops_sustained"] == "fallback"
+    peaks, kinds = bench.load_peaks(str(tmp_path / "absent.json"))
+    assert peaks == bench.FALLBACK_PEAKS and set(kinds.values()) == {"fallback"}
+    p.write_text("{not json")
+    assert bench.load_peaks(str(p))[0] == bench.FALLBACK_PEAKS
