@@ -56,6 +56,35 @@ def load_peaks(path=None):
     return peaks, kinds
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest value over all ranks (every rank calls this, in the same order); x itself
+    when no process group is running."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_ranks(flag: bool, device) -> bool:
+    """True only if `flag` holds on every rank (every rank calls this, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return bool(flag)
+    t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
+def whole_job_rate(work_per_rank: float, world: int, steps: int, elapsed_ms: float) -> float:
+    """Weak scaling: every rank does `work_per_rank` per step; the job's rate is all ranks' work
+    over the slowest rank's time."""
+    return work_per_rank * world * steps / (elapsed_ms * 1e-3)
+
+
 def workload_flops_bytes(tab, H, d, elt):
     from prefix_shared_attention_b200.metrics import algorithmic_bytes, algorithmic_flops
     return (algorithmic_flops(tab.prefix_len, tab.req_prefix, tab.suffix_len, H, d),
@@ -417,14 +446,11 @@ def main():
     elapsed_ms = t0.elapsed_time(t1)
     kernel_ms = [sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps)) / args.steps
                  for i in range(len(parts))]
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     ms_per_step = elapsed_ms / args.steps
-    value = step_flops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
-    req_s = tab.R * world * args.steps / (elapsed_ms * 1e-3)
+    value = whole_job_rate(step_flops, world, args.steps, elapsed_ms) / 1e12
+    req_s = whole_job_rate(tab.R, world, args.steps, elapsed_ms)
     peaks, peak_kinds = load_peaks()
     achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
     # Which roof binds: algorithmic FLOP per byte against the ridge of the measured peaks.
@@ -463,18 +489,15 @@ def main():
             host_ok = True
         free_now, _ = torch.cuda.mem_get_info()
         fits = free_now >= 0.9 * 2 * 4 * rows2 * row_b
-        if world > 1:
-            # Every rank takes the same collective steps: agree on whether all ranks run it.
-            flag = torch.tensor([1 if (host_ok and fits) else 0], device=dev)
-            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
-            host_ok, fits = bool(flag.item()) and host_ok, bool(flag.item()) and fits
-            if not (host_ok and fits):
-                host_ok = False
+        # Every rank takes the same collective steps: agree on whether all ranks run it.
+        everyone = all_ranks(host_ok and fits, dev)
         if not host_ok:
             e2e = {"value": None, "unit": UNIT,
                    "skipped": f"needs {need_host * local_world / 1e9:.0f} GB of pinned host memory on this node"}
         elif not fits:
             e2e = {"value": None, "unit": UNIT, "skipped": "two device buffer sets do not fit"}
+        elif not everyone:
+            e2e = {"value": None, "unit": UNIT, "skipped": "another rank cannot hold its end-to-end buffers"}
         else:
             plans2 = [bat.Plan(p.req_prefix, p.suffix_offsets, p.prefix_offsets, spec.H, spec.d, bat.BAT_BF16)
                       for p in parts2]
@@ -529,12 +552,8 @@ def main():
                     s_out.wait_event(ev)
             b_ev.record(s_out)
             torch.cuda.synchronize()
-            e_ms = a.elapsed_time(b_ev)
-            if world > 1:
-                tt = torch.tensor([e_ms], device=dev)
-                dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-                e_ms = float(tt.item())
-            e2e = {"value": step_flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+            e_ms = max_over_ranks(a.elapsed_time(b_ev), dev)
+            e2e = {"value": whole_job_rate(step_flops, world, args.e2e_steps, e_ms) / 1e12, "unit": UNIT,
                    "h2d_bytes_per_step": int(3 * tab.T_suf * row_b), "d2h_bytes_per_step": int(tab.T_suf * row_b),
                    "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
                    "pipeline": f"{len(parts2)} launches over 2 buffer sets; copy-in, forward, copy-out on 3 streams"}
