@@ -51,7 +51,9 @@ struct BoolC {
   static constexpr bool value = B;
 };
 
-__device__ uint32_t g_status_word;
+// Status words of this device: [0] bit 0 a wait timed out, bit 1 a debug check failed;
+// [1], [2] the first failed debug check and its value.
+__device__ uint32_t g_status_word[4];
 
 // Compile-time event trace of CTA 0 (off unless built with -DBAT_TRACE): per role, a list of
 // (code, clock64) pairs; code = event | x << 8 | index << 16.
@@ -104,11 +106,6 @@ __device__ unsigned* g_phase;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 2^8 between rescales
 constexpr int kItemQ = 4;                   // work items the producer may run ahead by
-#ifdef BAT_FMA_EXP_PAIRS
-constexpr int kFmaExpPairsSet = BAT_FMA_EXP_PAIRS;   // build-time override, same for every d
-#else
-constexpr int kFmaExpPairsSet = -1;
-#endif
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 // ------------------------------------------------------------------------------------
@@ -154,13 +151,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // Same test, but a thread whose phase is not complete is suspended (up to the hint, in ns)
 // until it completes, instead of returning at once: waiting warps then leave the issue slots
 // of their sub-partition to the warps that have work.
-__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -290,38 +287,6 @@ __device__ __forceinline__ void fadd2(float& a0, float& a1, float b0, float b1) 
       : "f"(b0), "f"(b1));
 }
 
-// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) on the packed fp32x2 FMA path.
-__device__ __forceinline__ void fma2v(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
-                                      float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-
-// 2^x for a pair, on the FMA pipe (offloads the MUFU).  Cody-Waite reduction: j = round(x)
-// by the 1.5 * 2^23 shifter, f = x - j in [-1/2, 1/2], 2^f by a degree-3 polynomial (relative
-// error 7.5e-5, coefficients from csrc/fit_exp2_poly.py), and 2^j added to the exponent
-// field.  x is clamped at -125 so the exponent field cannot underflow (2^-125 is 0 for every
-// use here: the row's largest term is >= 1).
-constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111251e-01f,
-                kExp2C3 = 5.517166480e-02f;
-__device__ __forceinline__ void exp2_fma2(float& x0, float& x1) {
-  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  float t0, t1, j0, j1, f0, f1, p0, p1;
-  fma2v(t0, t1, x0, x1, 1.f, 1.f, kShift, kShift);      // round to nearest integer in the low bits
-  fma2v(j0, j1, t0, t1, 1.f, 1.f, -kShift, -kShift);    // j = round(x)
-  fma2v(f0, f1, j0, j1, -1.f, -1.f, x0, x1);            // f = x - j
-  fma2v(p0, p1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
-  fma2v(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-  fma2v(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
-  x0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  x1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);
@@ -371,10 +336,6 @@ struct Cfg {
   // half of P, so the next tile's P can overwrite the first half early (measured faster at
   // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
   static constexpr int kPVHalves = D == 64 ? 2 : 1;
-  // Of every 8 score columns, pairs exponentiated on the FMA pipe (the rest on the MUFU).
-  // Measured no faster at either d (the exponential phase is not bound by MUFU throughput),
-  // so none by default; -DBAT_FMA_EXP_PAIRS=n selects n.
-  static constexpr int kFmaExpPairs = kFmaExpPairsSet >= 0 ? kFmaExpPairsSet : 0;
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return 128u * x; }
   __host__ __device__ static constexpr uint32_t o_col(int x) { return 256u + (uint32_t)D * x; }
@@ -387,7 +348,7 @@ struct Cfg {
   // same skip made the full-tile softmax slower, so it is off there.
   static constexpr bool kHalfSkip = D == 64;
   static constexpr uint32_t kIdescPV = make_idesc(128, D, true);
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * 4 + 4 * 2 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
+  static constexpr int kBarBytes = 8 * (3 * kStages + 2 * 4 + 4 * 2 + 2 + 2 * kItemQ) + 16 + 4 * kItemQ;
   static constexpr size_t kSmemBytes = 1024 + (size_t)(2 + kPBufs + kStages) * kTileBytes + kBarBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -481,8 +442,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   bool ok = mbar_test(bar, parity);
   if (!ok) {
     const uint64_t t0 = global_ns();
+    // One suspension never outlasts the wait's own limit (1 ms at most).
+    const uint32_t hint = c.limit_ns < 1000000ull ? (uint32_t)c.limit_ns : 1000000u;
     while (true) {
-      ok = mbar_test_suspend(bar, parity);
+      ok = mbar_test_suspend(bar, parity, hint);
       if (ok) break;
       if (*c.abort_flag) break;
       if (global_ns() - t0 > c.limit_ns) {
@@ -517,6 +480,7 @@ struct Smem {
   uint64_t* p_full;   // [2][2]: P of tile x, keys 64h .. 64h+63 written
   uint64_t* pv_done;  // [2][2]: PV of tile x over keys 64h .. 64h+63 done
   uint64_t* drain;    // [2]
+  uint64_t* v_zeroed;  // [kStages]: the tail rows of a ragged V tile in this slot are zeroed
   uint64_t* itq_full;   // [kItemQ]
   uint64_t* itq_empty;  // [kItemQ]
   volatile int* itq;    // [kItemQ] work-item indices handed from the producer to the others
@@ -569,11 +533,14 @@ __device__ __forceinline__ bool load_ring(const TcParams& p, const Smem<D>& sm, 
     if (!wait_bar(sm.kv_empty + s, ph ^ 1, ctl)) return false;
     if (lane == 0) {
       const CUtensorMap* m = from_cache ? (is_v ? &p.tm_vc : &p.tm_kc) : (is_v ? &p.tm_vs : &p.tm_ks);
+      int y = row0, x = w.head * D;
+      if (!BAT_DCHECK(p.status, y >= 0 && y < (from_cache ? (p.T_cache - p.chk_shrink) : (p.T_suf - p.chk_shrink)) && x >= 0 && x + D <= p.H * D,
+                      from_cache ? kChkCacheLoad : kChkSufLoad, y))
+        y = x = 0;
       mbar_expect_tx(sm.kv_full + s, C::kTileBytes);
 #pragma unroll
       for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, w.head * D + pn * 64, row0,
-                    sm.kv_full + s);
+        tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, x + pn * 64, y, sm.kv_full + s);
     }
     __syncwarp();
     ++ring;
@@ -614,18 +581,31 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
     ++kq;
     if (done) break;
     const WorkItem w = p.items[it];
+    if (lane == 0) {
+      // The item's fields stay inside the tensors (debug builds; the accesses are checked too).
+      BAT_DCHECK(p.status,
+                 w.head >= 0 && w.head < p.H && (w.n_q == 1 || w.n_q == 2) && w.qA_rows >= 1 && w.qA_rows <= kTileM &&
+                     w.qA_row0 >= 0 && w.qA_row0 + w.qA_rows <= (p.T_suf - p.chk_shrink) && w.sA_row0 >= 0 &&
+                     w.sA_row0 + w.sA_len <= (p.T_suf - p.chk_shrink) && w.pre_len >= 0 &&
+                     (w.pre_len == 0 || (w.pre_row0 >= 0 && w.pre_row0 + w.pre_len <= (p.T_cache - p.chk_shrink))) &&
+                     (w.n_q == 1 || (w.qB_rows >= 1 && w.qB_rows <= kTileM && w.qB_row0 >= 0 &&
+                                     w.qB_row0 + w.qB_rows <= (p.T_suf - p.chk_shrink) && w.sB_row0 >= 0 &&
+                                     w.sB_row0 + w.sB_len <= (p.T_suf - p.chk_shrink))) &&
+                     (w.split_slot < 0 || w.split_slot + w.n_q <= p.n_slots),
+                 kChkItem, it);
+    }
     BAT_TRACE_EV(0, tn, 1, 0, kq);
     for (int x = 0; ok && x < w.n_q; ++x) {
       ok = wait_bar(sm.q_empty + x, (qcnt[x] & 1) ^ 1, ctl);
       if (!ok) break;
       BAT_TRACE_EV(0, tn, 2, x, kq);
       if (lane == 0) {
+        int y = x ? w.qB_row0 : w.qA_row0, cx = w.head * D;
+        if (!BAT_DCHECK(p.status, y >= 0 && y < (p.T_suf - p.chk_shrink) && cx >= 0 && cx + D <= p.H * D, kChkQLoad, y)) y = cx = 0;
         mbar_expect_tx(sm.q_full + x, C::kTileBytes);
-        const int row0 = x ? w.qB_row0 : w.qA_row0;
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(sm.q + x * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q, w.head * D + pn * 64, row0,
-                      sm.q_full + x);
+          tma_load_2d(sm.q + x * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q, cx + pn * 64, y, sm.q_full + x);
       }
       __syncwarp();
       ++qcnt[x];
@@ -661,6 +641,24 @@ __device__ void vproducer_role(const TcParams& p, const Smem<D>& sm, const Ctl& 
   __syncwarp();
 }
 
+// Zeroes rows [valid, valid rounded up to 16) of a K/V tile in shared memory, in every
+// 64-column panel (one warp).  The 128-byte swizzle only permutes the 16-byte chunks within a
+// row, so a whole row is the same 128 bytes with or without it.  The writes are made visible
+// to the tensor core (async proxy) before the warp leaves.
+template <int D>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* tile, int valid) {
+  using C = Cfg<D>;
+  const int lane = threadIdx.x & 31;
+  const int n = (((valid + 15) & ~15) - valid) * C::kPanels * 8;   // 16-byte chunks
+  const uint32_t base = smem_u32(tile) + (uint32_t)valid * 128;
+  for (int i = lane; i < n; i += 32) {
+    const int rp = i >> 3;   // (row - valid) * kPanels + panel
+    st_shared_v4(base + (rp % C::kPanels) * C::kPanelBytes + (rp / C::kPanels) * 128 + (i & 7) * 16, 0u, 0u, 0u, 0u);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+}
+
 // MMA issuer of query tile X (warp 9 for A, warp 10 for B).  A single issuing thread would
 // serialise both tiles' bookkeeping against a tensor-core queue only about one instruction
 // deep; with one issuer per tile, one tile's waits and commits overlap the other's MMAs.
@@ -680,6 +678,7 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
   uint32_t ring = 0, vring = 0, qcnt = 0, s_issued = 0, p_seen = 0;
+  uint32_t vz_par = 0;   // bit s: parity of the next v_zeroed phase of ring slot s
   bool ok = true;
   int tn = 0;
   (void)tn;
@@ -767,8 +766,24 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         // the whole tile).  16 keys per instruction = two 8-row swizzle groups of V (2 KiB); LBO
         // steps between V's 64-column panels.
         const uint64_t vd = vdesc0 + (uint64_t)((s * C::kTileBytes) >> 4);
-        // P over keys 64 .. 127 of a tile with at most 64 valid keys is zero: skip those steps.
-        const int kk_end = (C::kHalfSkip && st.tile_valid(w, j) <= 64) ? 4 : 8;
+        // PV runs only over the 16-key steps that hold a valid key.  P is exactly 0 beyond
+        // `valid`, but the V rows there belong to other segments of the tensor (or were never
+        // written), and 0 * NaN = NaN would poison the whole output row; so the steps past the
+        // last valid key are not issued, and the rows between `valid` and the end of its
+        // 16-key step are zeroed in shared memory by exactly one issuer: the lower-numbered
+        // consumer of the tile, which the other consumer waits for.
+        const int valid = st.tile_valid(w, j);
+        const int kk_end = (valid + 15) >> 4;
+        if (valid & 15) {
+          if (X == ((mask & 1) ? 0 : 1)) {
+            zero_tail_rows<D>(sm.kv + s * C::kTileBytes, valid);
+            if (mask == 3 && lane == 0) mbar_arrive(sm.v_zeroed + s);
+          } else {
+            ok = wait_bar(sm.v_zeroed + s, (vz_par >> s) & 1, ctl);
+            if (!ok) break;
+          }
+          if (mask == 3) vz_par ^= 1u << s;
+        }
 #pragma unroll
         for (int h = 2 - C::kPVHalves; h < 2; ++h) {
           BAT_TRACE_EV(1 + X, tn, 3, X, p_seen);
@@ -911,8 +926,6 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         // Exponentials in two halves of 64 columns; each half is converted to bf16 pairs and
         // stored (TMEM or shared memory, asynchronously) while the next half's exponentials run.
-        // Of every eight columns, kFmaExpPairs pairs use the FMA-pipe exponential, the rest the
-        // MUFU.
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // A tile with at most 64 valid keys: keys 64 .. 127 carry no weight and PV skips them,
@@ -924,9 +937,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
 #pragma unroll
             for (int k = 0; k < 8; k += 2) ffma2(s[c + k], s[c + k + 1], s[c + k], s[c + k + 1], sl2, nm);
 #pragma unroll
-            for (int k = 0; k < 8 - 2 * C::kFmaExpPairs; ++k) s[c + k] = ex2(s[c + k]);
-#pragma unroll
-            for (int k = 8 - 2 * C::kFmaExpPairs; k < 8; k += 2) exp2_fma2(s[c + k], s[c + k + 1]);
+            for (int k = 0; k < 8; ++k) s[c + k] = ex2(s[c + k]);
             fadd2(a0, a1, s[c], s[c + 1]);
             fadd2(a2, a3, s[c + 2], s[c + 3]);
             fadd2(a0, a1, s[c + 4], s[c + 5]);
@@ -1014,20 +1025,26 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
         __syncwarp();
         if (lane == 0) {
           const int y = (X ? w.qB_row0 : w.qA_row0) + 32 * wq;
+          if (BAT_DCHECK(p.status, y >= 0 && y + 32 <= (p.T_suf - p.chk_shrink) && w.head >= 0 && w.head < p.H, kChkOutBulk, y)) {
 #pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_store_2d(&p.tm_o, sm.p + X * C::kTileBytes + pn * C::kPanelBytes + wq * 32 * 128, w.head * D + pn * 64, y);
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_store_2d(&p.tm_o, sm.p + X * C::kTileBytes + pn * C::kPanelBytes + wq * 32 * 128, w.head * D + pn * 64,
+                           y);
+          }
           bulk_commit();
         }
         o_pending = true;
         BAT_TRACE_EV(3 + X, tn, 14, X, s_seen);
-        if (p.lse) p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
+        if (p.lse && BAT_DCHECK(p.status, qrow >= 0 && qrow < (p.T_suf - p.chk_shrink) && w.head >= 0 && w.head < p.H, kChkLse, qrow))
+          p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
         o_stored = true;
       }
     }
     if (o_stored) {
     } else if (w.split_slot < 0) {
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)qrow * p.H + w.head) * D;
+      const bool row_ok =
+          !live || BAT_DCHECK(p.status, qrow >= 0 && qrow < (p.T_suf - p.chk_shrink) && w.head >= 0 && w.head < p.H, kChkOutRow, qrow);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -1036,22 +1053,23 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (live) {
+        if (live && row_ok) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
       BAT_TRACE_EV(3 + X, tn, 14, X, s_seen);
-      if (live && p.lse) p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
+      if (live && row_ok && p.lse) p.lse[(int64_t)w.head * p.T_suf + qrow] = lse2 * 0.69314718055994531f;
     } else {
       const int64_t slot = w.split_slot + X;
       float* dst = p.part_o + (slot * kTileM + row) * D;
+      const bool part_ok = !live || BAT_DCHECK(p.status, slot >= 0 && slot < p.n_slots, kChkPartial, slot);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
-        if (live) {
+        if (live && part_ok) {
           float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
@@ -1059,7 +1077,7 @@ __device__ void softmax_role(const TcParams& p, const Smem<D>& sm, const Ctl& ct
                                 __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
         }
       }
-      if (live) p.part_lse[slot * kTileM + row] = lse2;
+      if (live && part_ok) p.part_lse[slot * kTileM + row] = lse2;
     }
   }
   BAT_PHASE_FLUSH();
@@ -1089,7 +1107,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
   sm.p_full = sm.s_free + 2;
   sm.pv_done = sm.p_full + 4;
   sm.drain = sm.pv_done + 4;
-  sm.itq_full = sm.drain + 2;
+  sm.v_zeroed = sm.drain + 2;
+  sm.itq_full = sm.v_zeroed + C::kStages;
   sm.itq_empty = sm.itq_full + kItemQ;
   sm.itq = reinterpret_cast<volatile int*>(sm.itq_empty + kItemQ);
   sm.tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(sm.itq) + kItemQ);
@@ -1113,6 +1132,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     }
     mbar_init(sm.drain, 1);
     mbar_init(sm.drain + 1, 1);
+    for (int s = 0; s < C::kStages; ++s) mbar_init(sm.v_zeroed + s, 1);
     for (int i = 0; i < kItemQ; ++i) {
       mbar_init(sm.itq_full + i, 1);
       mbar_init(sm.itq_empty + i, C::kItemConsumers);

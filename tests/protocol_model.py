@@ -16,7 +16,10 @@ flight, the protocol has deadlocked.  The roles follow the kernel:
   mma X        walks the tiles in consumption order: S of key tile j+1 (K slot landed,
                Q landed for the first S, the softmax has read the previous S), then PV of
                tile j (V slot landed, P written, per P half); frees each slot by a commit or,
-               for a tile query tile X does not read, a plain arrive
+               for a tile query tile X does not read, a plain arrive.  A V tile whose valid
+               keys end inside a 16-key step has its tail rows zeroed by its lower-numbered
+               consumer, which arrives on the slot's v_zeroed barrier when both tiles read it;
+               the other consumer waits for that barrier
   softmax X    per tile: S landed -> s_free; optionally (data dependent) waits for the last
                PV before rescaling O; per P half: waits for the previous tile's PV of that
                half, writes P, p_full; after the item: waits for the last PV (epilogue)
@@ -70,6 +73,20 @@ class Stream:
         self.nsA = cd(w["sA_len"])
         self.nsB = 0 if self.shared else cd(w["sB_len"])
         self.n = self.npre + self.nsA + self.nsB
+        self.w = w
+
+    def valid(self, j):
+        """Valid keys of global tile j."""
+        w = self.w
+        if j < self.npre:
+            return min(TILE, int(w["pre_len"]) - j * TILE)
+        k = j - self.npre
+        if self.shared:
+            return min(TILE, int(w["sA_len"]) - k * TILE)
+        mm = min(self.nsA, self.nsB)
+        x = (k & 1) if k < 2 * mm else (0 if self.nsA > self.nsB else 1)
+        idx = (k >> 1) if k < 2 * mm else mm + (k - 2 * mm)
+        return min(TILE, int(w["sB_len" if x else "sA_len"]) - idx * TILE)
 
     def count(self, x):
         return self.npre + (self.nsA if (self.shared or x == 0) else self.nsB)
@@ -106,8 +123,10 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
     if two_rings:
         k_full, k_empty = ring("k", k_stages, 2)
         v_full, v_empty = ring("v", v_stages, 2)
+        v_zeroed = [Bar(f"v_zeroed{i}", 1) for i in range(v_stages)]
     else:
         kv_full, kv_empty = ring("kv", shared_stages, 2)
+        v_zeroed = [Bar(f"v_zeroed{i}", 1) for i in range(shared_stages)]
     bars = {n: [Bar(f"{n}{x}", c) for x in range(k)] for n, c, k in (
         ("q_full", 1, 2), ("q_empty", 1, 2), ("s_full", 1, 2), ("s_free", 128, 2), ("p_full", 128, 4),
         ("pv_done", 1, 4))}
@@ -179,6 +198,7 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
         q = mma_q[X]
         kr = vr = r = 0
         qcnt = s_issued = p_seen = 0
+        vz_par = [0] * len(v_zeroed)
         for ev in pop(1):
             if ev[0] != "item":
                 yield ev
@@ -194,12 +214,14 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
                 if two_rings:
                     if is_v:
                         f, e, ph = slot(vr, v_full, v_empty)
+                        zs = vr % len(v_full)
                         vr += 1
                     else:
                         f, e, ph = slot(kr, k_full, k_empty)
                         kr += 1
                 else:
                     f, e, ph = slot(r, kv_full, kv_empty)
+                    zs = r % len(kv_full)
                     r += 1
                 yield ("wait", f, ph)
                 if not mine or not ((st.mask(j) >> X) & 1):
@@ -219,6 +241,15 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
                     s_left -= 1
                     s_issued += 1
                 else:
+                    mask = st.mask(j)
+                    if st.valid(j) % 16:
+                        if X == (0 if mask & 1 else 1):
+                            if mask == 3:
+                                v_zeroed[zs].arrive()
+                        else:
+                            yield ("wait", v_zeroed[zs], vz_par[zs])
+                        if mask == 3:
+                            vz_par[zs] ^= 1
                     for h in range(2 - pv_halves, 2):
                         yield ("wait", bars["p_full"][2 * X + h], p_seen & 1)
                         q += [("mma",), ("commit", bars["pv_done"][2 * X + h])]

@@ -22,21 +22,50 @@ pytestmark = pytest.mark.gpu
 MAX_ABS = 2e-2
 MEAN_REL = 5e-3
 LSE_ABS = 2e-2
+# Guard rows around every output and LSE buffer: the kernels may write only inside the tensors
+# they are given, so the guards must hold their sentinel afterwards (a stand-in for a memory
+# checker, which is not available on the GPU pool).
+GUARD_ROWS = 128
+GUARD_VAL = -7.25
 
 
 def dcode(dtype):
     return bat.BAT_BF16 if dtype == "bf16" else bat.BAT_FP32
 
 
+def guarded(n_rows, row_shape, dtype, device):
+    """A buffer of n_rows rows (filled with NaN, so an unwritten row shows) between GUARD_ROWS
+    sentinel rows on each side; returns (whole buffer, view of the n_rows rows)."""
+    buf = torch.full((n_rows + 2 * GUARD_ROWS,) + tuple(row_shape), float("nan"), dtype=dtype, device=device)
+    buf[:GUARD_ROWS] = GUARD_VAL
+    buf[GUARD_ROWS + n_rows:] = GUARD_VAL
+    return buf, buf[GUARD_ROWS:GUARD_ROWS + n_rows]
+
+
+def assert_guards(buf, n_rows, what):
+    g = torch.cat([buf[:GUARD_ROWS].reshape(-1), buf[GUARD_ROWS + n_rows:].reshape(-1)])
+    assert bool((g == GUARD_VAL).all()), f"{what}: a kernel wrote outside the tensor it was given"
+
+
 def run_gpu(tab, xd, H, d, dtype, want_lse=True, scale=0.0, **plan_kw):
-    """xd: dict of device tensors. Returns (out, lse) device tensors."""
-    out = torch.full_like(xd["q"], float("nan"))
-    lse = torch.full((H, max(tab.T_suf, 1)), float("nan"), device=xd["q"].device) if want_lse else None
+    """xd: dict of device tensors. Returns (out, lse) device tensors; checks that nothing was
+    written into the guard rows around them."""
+    T = xd["q"].shape[0]
+    out_buf, out = guarded(T, xd["q"].shape[1:], xd["q"].dtype, xd["q"].device)
+    n_lse = H * max(tab.T_suf, 1)
+    if want_lse:
+        lse_buf, lse_flat = guarded(n_lse, (), torch.float32, xd["q"].device)
+        lse = lse_flat.view(H, max(tab.T_suf, 1))
+    else:
+        lse = None
     with bat.Plan(tab.req_prefix, tab.suffix_offsets, tab.prefix_offsets, H, d, dcode(dtype), **plan_kw) as plan:
         bat.bat_attention_forward(plan, xd["q"], xd["k_suf"], xd["v_suf"], xd["k_cache"], xd["v_cache"], out=out,
                                   lse=lse, scale=scale)
         st = bat.bat_get_device_status()
     assert st == bat.BAT_OK, bat.last_error()
+    assert_guards(out_buf, T, "out")
+    if want_lse:
+        assert_guards(lse_buf, n_lse, "lse")
     return out, lse
 
 
@@ -213,10 +242,58 @@ def test_wait_timeout_reports_and_context_survives():
             st = bat.bat_get_device_status()
     finally:
         bat.bat_set_wait_timeout_ns(0)
-    assert st in (bat.BAT_ERR_TIMEOUT, bat.BAT_OK)
+    # With a 1 ns limit the first wait whose phase has not completed yet expires (the softmax
+    # waits for an S that the tensor core cannot have finished when it first looks), so the
+    # abort path must have run and reported.
+    assert st == bat.BAT_ERR_TIMEOUT, f"expected BAT_ERR_TIMEOUT, got {st}: {bat.last_error()}"
     # The context stays usable and the next run is correct.
     full_parity(tab, 2, 128, "bf16", 9)
     assert bat.bat_get_device_status() == bat.BAT_OK
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 64), ("bf16", 128), ("fp32", 64)])
+@pytest.mark.parametrize("split", [0, 2])
+def test_nan_neighbour_rows(dtype, d, split):
+    """Rows that a tile window reaches beyond its segment may hold anything, NaN included:
+    cache slots reserved but not yet built (allocated uninitialised), or another request's
+    garbage tokens.  Masked keys must weigh exactly 0 there, so every other request's output
+    stays exact.  Lead page (Bat), section "This paper's idea": the prefix K/V is computed once
+    and kept in a pool that many requests read, so one bad slot must not reach them."""
+    # Pool: referenced prefixes (even ids) interleaved with unreferenced NaN slots (odd ids),
+    # one NaN slot after the last prefix; lengths end inside a 16-key step.
+    pre = np.array([37, 21, 201, 7, 99, 300, 130, 50, 1, 19])
+    nan_pre = [1, 3, 5, 7, 9]
+    req = np.array([0, 0, 2, 4, 6, 2, -1, 4, 6, 0, 8, 2], np.int32)
+    suf = np.array([45, 130, 77, 1, 257, 19, 100, 128, 33, 200, 70, 131])
+    poisoned = [5, 8]                       # requests whose own q/k/v rows are NaN
+    tab = RequestTable(pre, req, suf)
+    po, so = tab.prefix_offsets, tab.suffix_offsets
+
+    def mutate(x):
+        for p in nan_pre:
+            x["k_cache"][po[p]:po[p + 1]] = float("nan")
+            x["v_cache"][po[p]:po[p + 1]] = float("nan")
+        for r in poisoned:
+            for k in ("q", "k_suf", "v_suf"):
+                x[k][so[r]:so[r + 1]] = float("nan")
+
+    H = 2
+    x = host_tensors(tab, H, d, dtype, 31)
+    mutate(x)
+    xd = {k: v.cuda() for k, v in x.items()}
+    out, lse = run_gpu(tab, xd, H, d, dtype, split_mode=split, split_chunk_tiles=1 if split else 0)
+    ref_o, ref_l = oracle.bipartite_attention(x["q"], x["k_suf"], x["v_suf"], x["k_cache"], x["v_cache"], po, so,
+                                              tab.req_prefix)
+    keep = np.ones(tab.T_suf, bool)
+    for r in poisoned:
+        keep[so[r]:so[r + 1]] = False
+    assert np.isfinite(ref_o[keep]).all()
+    o = out.float().cpu().double().numpy()
+    assert np.isfinite(o[keep]).all(), "a NaN in a masked row leaked into another request's output"
+    mx, mr = errors(o[keep], ref_o[keep])
+    assert mx <= MAX_ABS and mr <= MEAN_REL, (mx, mr)
+    lmx = float(np.abs(lse.cpu().double().numpy()[:, keep] - ref_l[:, keep]).max())
+    assert lmx <= LSE_ABS, lmx
 
 
 # --------------------------------------------------------------------------------------
@@ -255,11 +332,47 @@ def test_long_user_history_sampled():
     sampled_parity("long-user-history", 16)
 
 
-def test_mixed_sampled_one_launch():
+def mixed_sample(sub_tab, per_kind, rng):
+    """Requests of one launch to check: `per_kind` of each prefix kind (user block cached /
+    item block cached), drawn at random, plus the heaviest request of the launch (longest
+    prefix + suffix: the deepest key stream and rescale chain)."""
+    Lp = sub_tab.prefix_len_of_request()
+    pick = [int(np.argmax(Lp + sub_tab.suffix_len))]
+    for k in (0, 1):
+        idx = np.flatnonzero(sub_tab.kind == k)
+        pick += [int(i) for i in rng.choice(idx, size=min(per_kind, len(idx)), replace=False)]
+    return np.unique(np.array(pick, np.int64))
+
+
+def test_mixed_sampled_every_launch():
+    """The mixed batch in the launch configuration the bench times (8 request-disjoint launches
+    over one resident prefix cache): from every launch, 16 user-prefix and 16 item-prefix
+    requests plus the launch's heaviest request, 264 in all, against the oracle."""
     free, _ = torch.cuda.mem_get_info()
     if free < 150e9:
         pytest.skip(f"needs ~140 GB free device memory, {free / 1e9:.0f} GB free")
-    sampled_parity("mixed", 24, launch=3, n_launches=8)
+    name = "mixed"
+    spec = CONFIGS[name]
+    tab = make_table(name)
+    parts = split_launches(tab, 8)
+    cache = device_tensors(tab, spec.H, spec.d, spec.dtype, spec.seed + 17, which=("k_cache", "v_cache"))
+    rng = np.random.default_rng(123)
+    checked = 0
+    for i, part in enumerate(parts):
+        xd = dict(cache)
+        xd.update(device_tensors(part, spec.H, spec.d, spec.dtype, spec.seed + 100 + i, which=("q", "k_suf", "v_suf")))
+        out, lse = run_gpu(part, xd, spec.H, spec.d, spec.dtype)
+        reqs = mixed_sample(part, 16, rng)
+        sub, host, rows = gather_requests(part, xd, reqs, out=out)
+        lse_rows = lse[:, torch.from_numpy(rows).cuda()].cpu()
+        ref_o, ref_l = oracle.bipartite_attention(host["q"], host["k_suf"], host["v_suf"], host["k_cache"],
+                                                  host["v_cache"], sub.prefix_offsets, sub.suffix_offsets,
+                                                  sub.req_prefix)
+        assert_parity(host["out"], lse_rows, ref_o, ref_l, f"{name} launch {i}")
+        checked += len(reqs)
+        del xd, out, lse
+        torch.cuda.empty_cache()
+    assert checked >= 8 * 33
 
 
 # --------------------------------------------------------------------------------------

@@ -72,3 +72,27 @@ def test_model_detects_a_missing_release():
     finally:
         pm.Bar = orig
     assert r.startswith("deadlock") and "v_empty" in r
+
+
+def test_model_needs_the_zeroed_hand_off():
+    """The second consumer of a ragged V tile really waits for the first one's zeroing: if the
+    zeroing issuer never signals, the model deadlocks on v_zeroed."""
+    import protocol_model as pm
+
+    class NoZeroed(pm.Bar):
+        def arrive(self, n=1):
+            if "v_zeroed" in self.name:
+                return
+            super().arrive(n)
+
+    # One prefix of 600 keys (last tile holds 88: not a multiple of 16) read by two requests.
+    items = work_items(RequestTable(np.array([600]), np.array([0, 0], np.int32), np.array([256, 256])))
+    assert any(int(w["n_q"]) == 2 for w in items)
+    orig = pm.Bar
+    pm.Bar = NoZeroed
+    try:
+        results = [pm.simulate(items, *cfg, seed=5) for cfg in (KERNEL_D128, KERNEL_D64)]
+    finally:
+        pm.Bar = orig
+    for r in results:
+        assert r.startswith("deadlock") and "v_zeroed" in r, r
