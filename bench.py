@@ -29,7 +29,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, gather_requests, host_tensors, make_table, split_launches  # noqa: E402
+from workloads import CONFIGS, device_tensors, host_tensors, make_table, split_launches  # noqa: E402
 
 METRIC = "bipartite-attention TFLOP/s and requests/s on 1 B200; % of bf16 tensor roofline"
 UNIT = "TFLOP/s"
@@ -313,6 +313,16 @@ def cpu_baseline(workload, target_s=12.0, prefix_side=False):
             "requests_per_s": n / dt}
 
 
+def repo_libraries_loaded():
+    """Shared objects of this repository mapped into the process (the reference arm must map
+    none: it times the oracle alone)."""
+    try:
+        maps = open("/proc/self/maps").read().splitlines()
+    except OSError:
+        return []
+    return sorted({l.split()[-1] for l in maps if l.split()[-1].startswith(ROOT) and ".so" in l.split()[-1]})
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -335,13 +345,74 @@ def run_reference(args, rank, world):
             "requests_per_s": n * args.steps / dt,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{n} of {tab.R} requests per step, fp64 numpy oracle"},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "repo_libraries_loaded": [os.path.relpath(p, ROOT) for p in repo_libraries_loaded()]}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # --------------------------------------------------------------------------------------------
 # GPU arm
+
+SECONDARY = ("long-user-history", "item-as-prefix", "user-as-prefix")
+
+
+def roofline_of(flops, nbytes, kernel_s, peaks):
+    """Which roof binds (algorithmic FLOP per byte against the ridge of the measured peaks) and
+    the fraction of it reached; tensor-bound work is compared with the burst bf16 figure."""
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    tf = flops / kernel_s / 1e12
+    if flops / nbytes < ridge:
+        gbs = nbytes / kernel_s / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": gbs / float(peaks["hbm_gbs"]), "tensor_tflops": tf}
+    return {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+            "frac": tf / float(peaks["bf16_tflops"])}
+
+
+def time_secondary(name, dev, peaks, reps=10, warmup=3):
+    """CUDA-event time of one forward of a named workload (one launch), L2 flushed before every
+    timed launch, clocks sampled meanwhile.  The same kernel and launch path as the main line."""
+    import torch
+    import prefix_shared_attention_b200 as bat
+    spec = CONFIGS[name]
+    tab = make_table(name)
+    x = device_tensors(tab, spec.H, spec.d, spec.dtype, spec.seed, device=dev)
+    out = torch.empty_like(x["q"])
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    with bat.Plan(tab.req_prefix, tab.suffix_offsets, tab.prefix_offsets, spec.H, spec.d, bat.BAT_BF16) as plan:
+        ws = torch.empty(max(plan.workspace_bytes, 16), dtype=torch.uint8, device=dev)
+
+        def fwd():
+            bat.bat_attention_forward(plan, x["q"], x["k_suf"], x["v_suf"], x["k_cache"], x["v_cache"], out=out,
+                                      workspace=ws, stream=stream)
+        for _ in range(warmup):
+            fwd()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        clocks = clock_sampler(dev.index)
+        clocks.start()
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fwd()
+            b.record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        if bat.bat_get_device_status() != bat.BAT_OK:
+            raise RuntimeError(bat.last_error())
+        n_launch = 1 + (plan.info().n_merges > 0)
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ms[len(ms) // 2]
+    flops, nbytes = workload_flops_bytes(tab, spec.H, spec.d, 2)
+    r = {"tflops": flops / (med * 1e-3) / 1e12, "requests_per_s": tab.R / (med * 1e-3), "ms": med,
+         "launches": n_launch, "reps": reps, "l2": "flushed before every timed launch",
+         "roofline": roofline_of(flops, nbytes, med * 1e-3, peaks), "clocks": clk}
+    del x, out, flush, ws
+    torch.cuda.empty_cache()
+    return r
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -359,6 +430,8 @@ def main():
                          "its own tokens (the outputs of the prefix tokens themselves)")
     ap.add_argument("--subset", type=int, default=0,
                     help="profiling aid: only the first N requests (and the prefixes they read); not a bench line")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the one-launch timings of the other bf16 workloads")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("BAT_BENCH_ALLOW_SHORT"), \
         "at least 3 warm-up steps"
@@ -393,7 +466,6 @@ def main():
     parts = split_launches(tab, n_launch)
     seed = spec.seed + 1000 * rank
 
-    from workloads import device_tensors
     cache = device_tensors(tab, spec.H, spec.d, spec.dtype, seed, device=dev, which=("k_cache", "v_cache"))
     rows = max(p.T_suf for p in parts)
     suf = device_tensors(parts[0], spec.H, spec.d, spec.dtype, seed + 1, device=dev, which=("q", "k_suf", "v_suf"),
@@ -456,11 +528,10 @@ def main():
     # Which roof binds: algorithmic FLOP per byte against the ridge of the measured peaks.
     ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
     hbm_bound = step_flops / step_bytes < ridge
-    # The denominator follows how long the kernel holds the tensor pipe: a timed region of a
-    # second or more runs under the board's power cap like the sustained GEMM measurement
-    # (seconds back to back), a shorter one is compared with the burst figure.
-    sustained = elapsed_ms >= 1000.0 and "bf16_tflops_sustained" in peaks
-    peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
+    # The fraction divides by the burst bf16 GEMM figure, the denominator the target is stated
+    # against (>= 60 % of it); the sustained figure (the same GEMM back to back for seconds,
+    # under the power cap) is reported beside it.
+    peak = float(peaks["bf16_tflops"])
     kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
     traffic = None if args.prefix_side else traffic_per_launch(args.workload, kernel_src)
 
@@ -566,10 +637,15 @@ def main():
         for pl in plans:
             pl.close()
 
+    suf = cache = out = ws = None
+    torch.cuda.empty_cache()
+    secondary = None
+    if not (args.no_secondary or args.subset or args.prefix_side or args.workload != "mixed"):
+        # One launch of each other bf16 workload, on every rank (same steps everywhere).
+        secondary = {name: time_secondary(name, dev, load_peaks()[0]) for name in SECONDARY}
+
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        suf = cache = out = ws = None
-        torch.cuda.empty_cache()
         base = cpu_baseline(args.workload, prefix_side=args.prefix_side)
 
     if rank == 0:
@@ -586,9 +662,8 @@ def main():
             "plan_ms": plan_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": (f"{peak_kinds['bf16_tflops_sustained']} bf16_tflops_sustained (timed region "
-                                         f"{elapsed_ms / 1e3:.1f} s under the power cap)" if sustained
-                                         else f"{peak_kinds['bf16_tflops']} bf16_tflops (burst)"),
+                         "peak_source": f"{peak_kinds['bf16_tflops']} bf16_tflops (burst)",
+                         "target_frac": 0.60, "target_met": achieved / peak >= 0.60,
                          "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                          "frac_of_spec": achieved / 2250.0,
@@ -598,6 +673,8 @@ def main():
                          "alg_gb_per_launch": [b / 1e9 for b in bytes_l]},
             "cpu_baseline": base, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
         }
+        if secondary is not None:
+            line["secondary"] = secondary
         if hbm_bound:
             # Left of the ridge: the bandwidth roof binds; report against the measured copy rate.
             gbs = step_bytes / (sum(kernel_ms) * 1e-3) / 1e9

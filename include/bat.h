@@ -40,7 +40,8 @@ typedef enum {
   BAT_ERR_UNSUPPORTED = 2, /* valid arguments the library does not implement (e.g. bf16 d=32) */
   BAT_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
   BAT_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait and returned early */
-  BAT_ERR_OOM = 5          /* a host or device allocation of the library failed */
+  BAT_ERR_OOM = 5,         /* a host or device allocation of the library failed */
+  BAT_ERR_DEVICE_CHECK = 6 /* debug builds only: a device-side bounds check failed */
 } bat_status;
 
 typedef enum { BAT_BF16 = 0, BAT_FP32 = 1 } bat_dtype;
@@ -88,10 +89,15 @@ bat_status bat_prefix_kv_build(const void* k_src, const void* v_src, const int64
 
 /*
  * bat_plan_create - host grouping pass over one batch of requests.
+ * Lead page (Bat), section "Why it works": a hot item's cached K/V serves every user who sees
+ * it and a user's cached K/V serves all of that user's requests, so the requests that read one
+ * prefix are batched together and its K/V is streamed once for all of them.
  * Buckets the requests by the prefix they read, pairs their 128-row query tiles into work
  * items that stream each prefix's K/V tiles once, orders the items heaviest group first,
  * optionally splits over-long key streams (partials merged by log-sum-exp), and uploads the
  * work list to the current device on `stream` (the plan owns that device memory).
+ * `dt` and `opts` go beyond the minimal interface (the pages give none): the dtype fixes
+ * which kernel the plan is for, and the options expose the split policy and a host-only mode.
  *   req_prefix      HOST int32 [R]; prefix id in [0, P) or -1 for none
  *   suffix_offsets  HOST int64 [R+1]; request r owns suffix rows [so[r], so[r+1])
  *   prefix_offsets  HOST int64 [P+1]; prefix p owns cache rows [po[p], po[p+1])
@@ -145,7 +151,10 @@ bat_status bat_plan_merges(const bat_plan* plan, void* dst, size_t dst_bytes);
 
 /*
  * bat_attention_forward - the hot path: bipartite prefix-shared attention for every
- * suffix row of the plan's requests.
+ * suffix row of the plan's requests.  Lead page (Bat), sections "This paper's idea" and
+ * "Why it works": each request's own tokens attend, with no mask, over the cached K/V of
+ * its prefix block followed by its own K/V; the result equals full bidirectional attention
+ * over the whole request, whichever block is the prefix.
  *   q, k_suf, v_suf   device [T_suf, H, d] of dtype dt: each request's own tokens
  *   k_cache, v_cache  device [T_cache, H, d] of dtype dt: the prefix pool (may be NULL
  *                     when T_cache = 0)
@@ -154,8 +163,13 @@ bat_status bat_plan_merges(const bat_plan* plan, void* dst, size_t dst_bytes);
  *   lse               device fp32 [H, T_suf] or NULL: natural-log log-sum-exp of the
  *                     scaled scores of each row
  *   workspace         device scratch of at least bat_workspace_bytes(plan) bytes (NULL if 0)
- * Every row of the K/V tensors that a 128-row tile window can reach must hold finite values:
- * the kernel loads whole tiles and weights rows outside a segment by exactly 0.
+ * Rows outside a request's or a prefix's segment are never weighted: the kernel loads whole
+ * 128-row tiles, but keys beyond a segment get weight exactly 0 and their V rows are never
+ * multiplied in, so such rows may hold anything (NaN included: an unbuilt pool slot, or another
+ * request's garbage) without reaching other rows' outputs.
+ * One plan runs on one stream at a time: the plan holds the kernel's work-item counter, which
+ * each call resets on `stream`, so two calls with the same plan whose kernels overlap (on two
+ * streams) would share it and skip or repeat work.  Use one plan per concurrent stream.
  * Asynchronous on `stream`.  Device-side wait timeouts are reported by
  * bat_get_device_status.
  * Errors: BAT_ERR_INVALID_ARG (null/misaligned pointer, dtype/d differ from the plan's,
@@ -180,7 +194,9 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
  *     it, so issue them on one stream.  It keeps the previous call's contents; nothing in it
  *     needs to start at zero.
  *   - The first call on each device resolves the array's address (with that device current);
- *     make it before any stream capture starts on that device.
+ *     make it before any stream capture starts on that device.  The address is kept for the
+ *     life of the process: after cudaDeviceReset (which unloads the library's device code) it
+ *     is stale, so do not call this entry point again on a device that was reset.
  * Errors: those of bat_attention_forward, plus BAT_ERR_CUDA if the address lookup fails.
  */
 bat_status bat_attention_forward_noalloc(const bat_plan* plan, const void* q, const void* k_suf,
@@ -189,8 +205,9 @@ bat_status bat_attention_forward_noalloc(const bat_plan* plan, const void* q, co
                                          void* stream);
 
 /* Synchronises `stream`, then reports and clears the device-side status word of the
- * current device: BAT_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last call,
- * BAT_ERR_CUDA on a CUDA error, else BAT_OK. */
+ * current device: BAT_ERR_DEVICE_CHECK if a bounds check of a debug build failed (the message
+ * names the check and the offending value), BAT_ERR_TIMEOUT if a kernel abandoned a bounded
+ * wait since the last call, BAT_ERR_CUDA on a CUDA error, else BAT_OK. */
 bat_status bat_get_device_status(void* stream);
 
 /* Upper bound, in nanoseconds, on every spin-wait inside the kernels (default 2e9).
@@ -202,6 +219,16 @@ const char* bat_last_error(void);
 
 /* ABI version: (major << 16) | minor. */
 int32_t bat_version(void);
+
+/* 1 in the debug build (libbat_debug.so, compiled with -DBAT_DEBUG), whose kernels check every
+ * tensor-map coordinate and store index against the tensors' bounds before using it: a failed
+ * check records its code and value in the device status word (reported by
+ * bat_get_device_status as BAT_ERR_DEVICE_CHECK) and the access is skipped (stores) or clamped
+ * into the tensor (loads).  No check traps.  0 in the normal build, which has no checks.
+ * In the debug build only, the environment variable BAT_DEBUG_SHRINK_BOUNDS=n makes the checks
+ * treat every tensor as n rows shorter than it is (the accesses themselves are unchanged and
+ * stay inside the real tensors): a negative control showing that the checks fire. */
+int32_t bat_debug_checks(void);
 
 #ifdef __cplusplus
 }

@@ -14,11 +14,14 @@ from typing import Optional
 
 import numpy as np
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbat.so")
+# The library this process uses: the in-tree libbat.so, or the file BAT_LIBRARY names (the
+# debug build, libbat_debug.so, whose kernels check their bounds).
+LIB_PATH = os.environ.get("BAT_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbat.so")
 
-BAT_OK, BAT_ERR_INVALID_ARG, BAT_ERR_UNSUPPORTED, BAT_ERR_CUDA, BAT_ERR_TIMEOUT, BAT_ERR_OOM = range(6)
+(BAT_OK, BAT_ERR_INVALID_ARG, BAT_ERR_UNSUPPORTED, BAT_ERR_CUDA, BAT_ERR_TIMEOUT, BAT_ERR_OOM,
+ BAT_ERR_DEVICE_CHECK) = range(7)
 STATUS_NAMES = {0: "BAT_OK", 1: "BAT_ERR_INVALID_ARG", 2: "BAT_ERR_UNSUPPORTED", 3: "BAT_ERR_CUDA",
-                4: "BAT_ERR_TIMEOUT", 5: "BAT_ERR_OOM"}
+                4: "BAT_ERR_TIMEOUT", 5: "BAT_ERR_OOM", 6: "BAT_ERR_DEVICE_CHECK"}
 BAT_BF16, BAT_FP32 = 0, 1
 
 
@@ -65,6 +68,7 @@ _SIGNATURES = {
     "bat_set_wait_timeout_ns": (_i32, [_u64]),
     "bat_last_error": (C.c_char_p, []),
     "bat_version": (_i32, []),
+    "bat_debug_checks": (_i32, []),
 }
 
 
@@ -268,3 +272,7 @@ def bat_set_wait_timeout_ns(ns: int) -> None:
 
 def bat_version() -> int:
     return int(lib.bat_version())
+
+
+def bat_debug_checks() -> bool:
+    return bool(lib.bat_debug_checks())

@@ -1,11 +1,16 @@
 """Build libbat.so in-tree for sm_100a.
 
-    python -m prefix_shared_attention_b200.build [--force] [--verbose]
+    python -m prefix_shared_attention_b200.build [--force] [--verbose] [--debug]
 
 Every CUDA source is compiled with nvcc for ``sm_100a`` only (tcgen05, TMA) and linked
 with the static CUDA runtime into ``prefix_shared_attention_b200/libbat.so``.  Objects go
 to ``prefix_shared_attention_b200/_build/``.  Sources newer than the library trigger a
 rebuild of their object.
+
+``--debug`` builds ``libbat_debug.so`` instead (objects in ``_build_debug/``), compiled with
+``-DBAT_DEBUG``: its kernels check every tensor-map coordinate and store index against the
+tensors' bounds and report a failed check through the device status word (no check traps).
+Select it at run time with ``BAT_LIBRARY=<path to libbat_debug.so>``.
 """
 
 from __future__ import annotations
@@ -23,6 +28,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libbat.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libbat_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-I", INCLUDE, "-I", CSRC,
@@ -49,19 +56,21 @@ def _mtime(p):
     return os.path.getmtime(p) if os.path.exists(p) else -1.0
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    flags = FLAGS + (["-DBAT_DEBUG"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     newest_header = max(_mtime(h) for h in headers())
     jobs = []
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or _mtime(obj) < max(_mtime(src), newest_header):
-            cmd = [cc] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
+            cmd = [cc] + ARCH + flags + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
             if src.endswith(".cpp"):
-                cmd = [cc] + FLAGS + ["-x", "c++", "-c", src, "-o", obj]
+                cmd = [cc] + flags + ["-x", "c++", "-c", src, "-o", obj]
             jobs.append(cmd)
 
     def run(cmd):
@@ -75,12 +84,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
 
     with ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
         list(ex.map(run, jobs))
-    if force or jobs or _mtime(LIB) < max(_mtime(o) for o in objs):
-        tmp = LIB + ".tmp"
+    if force or jobs or _mtime(lib) < max(_mtime(o) for o in objs):
+        tmp = lib + ".tmp"
         cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + ["-lpthread", "-ldl", "-lrt"]
         run(cmd)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 def main():
@@ -88,8 +97,9 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libbat_debug.so (device-side bounds checks)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_verbose))
+    print(build(a.force, a.verbose, a.ptxas_verbose, a.debug))
 
 
 if __name__ == "__main__":

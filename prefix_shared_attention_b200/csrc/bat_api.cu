@@ -91,6 +91,18 @@ bat_status encode_map(CUtensorMap* m, const void* base, int64_t T, int32_t H, in
   return BAT_OK;
 }
 
+// Debug builds only: BAT_DEBUG_SHRINK_BOUNDS=n makes the device-side checks treat every tensor
+// as n rows shorter than it is, so a valid run trips them on its last rows while every access
+// the kernels still make stays inside the real tensors (a negative control of the checks).
+int32_t debug_shrink() {
+#ifdef BAT_DEBUG
+  const char* e = getenv("BAT_DEBUG_SHRINK_BOUNDS");
+  return e ? atoi(e) : 0;
+#else
+  return 0;
+#endif
+}
+
 }  // namespace
 
 namespace bat {
@@ -102,7 +114,15 @@ extern "C" {
 
 const char* bat_last_error(void) { return g_err.c_str(); }
 
-int32_t bat_version(void) { return (1 << 16) | 0; }
+int32_t bat_version(void) { return (1 << 16) | 1; }
+
+int32_t bat_debug_checks(void) {
+#ifdef BAT_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 bat_status bat_set_wait_timeout_ns(uint64_t ns) {
   g_wait_ns.store(ns ? ns : kDefaultWaitNs);
@@ -368,6 +388,9 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
     p.status = status;
     p.wait_ns = g_wait_ns.load();
     p.item_counter = plan->d_counter;
+    p.T_cache = (int32_t)(has_cache ? plan->T_cache : plan->T_suf);
+    p.n_slots = (int32_t)plan->host.n_slots;
+    p.chk_shrink = debug_shrink();
     e = cudaMemsetAsync(plan->d_counter, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return cuda_fail(e, "resetting the work-item counter");
     const int grid = (int)std::min<int64_t>(plan->host.n_items, plan->num_sms);
@@ -390,6 +413,10 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
     p.T_suf = (int32_t)plan->T_suf;
     p.H = plan->H;
     p.scale = sc;
+    p.T_cache = (int32_t)plan->T_cache;
+    p.n_slots = (int32_t)plan->host.n_slots;
+    p.status = status;
+    p.chk_shrink = debug_shrink();
     e = bat::launch_attn_simt(plan->d, p, s);
     if (e != cudaSuccess) return cuda_fail(e, "fp32 attention kernel launch");
   }
@@ -403,6 +430,9 @@ bat_status bat_attention_forward(const bat_plan* plan, const void* q, const void
     m.lse = lse;
     m.T_suf = (int32_t)plan->T_suf;
     m.H = plan->H;
+    m.n_slots = (int32_t)plan->host.n_slots;
+    m.status = status;
+    m.chk_shrink = debug_shrink();
     e = bat::launch_merge(plan->d, dt == BAT_BF16, m, s);
     if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
   }
@@ -416,13 +446,17 @@ bat_status bat_get_device_status(void* stream) {
   uint32_t* word = nullptr;
   e = bat::device_status_word(&word);
   if (e != cudaSuccess) return cuda_fail(e, "device status word");
-  uint32_t v = 0;
-  e = cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost);
+  uint32_t v[3] = {0, 0, 0};
+  e = cudaMemcpy(v, word, sizeof(v), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-  if (v) {
+  if (v[0]) {
     e = cudaMemset(word, 0, sizeof(v));
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
-    return fail(BAT_ERR_TIMEOUT, "a kernel abandoned a bounded wait (status 0x%x); its outputs are incomplete", v);
+    if (v[0] & 2u)
+      return fail(BAT_ERR_DEVICE_CHECK,
+                  "a device-side bounds check failed (check %u, value %u; status 0x%x); the access was skipped",
+                  v[1], v[2], v[0]);
+    return fail(BAT_ERR_TIMEOUT, "a kernel abandoned a bounded wait (status 0x%x); its outputs are incomplete", v[0]);
   }
   return BAT_OK;
 }

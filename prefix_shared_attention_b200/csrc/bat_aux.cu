@@ -33,6 +33,14 @@ __global__ void __launch_bounds__(128) bat_attn_simt_kernel(const SimtParams p) 
   const int s_len = own_a ? w.sA_len : w.sB_len;
   const int64_t row_stride = (int64_t)p.H * D;
   const int64_t col = (int64_t)w.head * D + lane * E;
+  // Debug builds: every row this query tile reads or writes lies inside its tensor.
+  if (!BAT_DCHECK(p.status,
+                  w.head >= 0 && w.head < p.H && rows >= 0 && rows <= kTileM && q0 >= 0 && q0 + rows <= (p.T_suf - p.chk_shrink) &&
+                      s_row0 >= 0 && s_row0 + s_len <= (p.T_suf - p.chk_shrink) &&
+                      (w.pre_len == 0 || (w.pre_row0 >= 0 && w.pre_row0 + w.pre_len <= (p.T_cache - p.chk_shrink))) &&
+                      (w.split_slot < 0 || (w.split_slot >= 0 && w.split_slot + X < p.n_slots)),
+                  kChkSimtRow, blockIdx.x))
+    return;
   for (int r = warp; r < rows; r += 4) {
     float q[E], o[E];
 #pragma unroll
@@ -93,6 +101,14 @@ template <typename OutT, int D>
 __global__ void __launch_bounds__(256) bat_merge_kernel(const MergeParams p) {
   const MergeJob j = p.jobs[blockIdx.x];
   constexpr int C4 = D / 4;
+  // Debug builds: every partial it reads and every row it writes lies inside its buffer.
+  if (!BAT_DCHECK(p.status,
+                  j.n_chunks >= 1 && j.slot0 >= 0 && j.slot_stride >= 0 &&
+                      j.slot0 + (int64_t)(j.n_chunks - 1) * j.slot_stride < p.n_slots && j.q_rows >= 0 &&
+                      j.q_rows <= kTileM && j.q_row0 >= 0 && j.q_row0 + j.q_rows <= (p.T_suf - p.chk_shrink) && j.head >= 0 &&
+                      j.head < p.H,
+                  kChkMerge, blockIdx.x))
+    return;
   for (int idx = threadIdx.x; idx < j.q_rows * C4; idx += blockDim.x) {
     const int r = idx / C4, c4 = idx % C4;
     float mx = -INFINITY;

@@ -8,6 +8,36 @@
 
 namespace bat {
 
+// Device-side bounds checks of debug builds (-DBAT_DEBUG; the library is then libbat_debug.so).
+// A failed check sets bit 1 of the device status word, records the check's code and the
+// offending value in words 1 and 2 (the first failure wins), and the caller skips the access
+// (stores) or clamps it into the tensor (loads, so every barrier still completes).  Nothing
+// traps.  In normal builds a check is the constant `true` and costs nothing.
+enum DebugCheck : uint32_t {
+  kChkQLoad = 1,      // Q tile coordinates inside q
+  kChkCacheLoad = 2,  // K/V tile coordinates inside the cache
+  kChkSufLoad = 3,    // K/V tile coordinates inside k_suf / v_suf
+  kChkOutBulk = 4,    // bulk store of 32 output rows inside out
+  kChkOutRow = 5,     // one output row inside out
+  kChkLse = 6,        // LSE element inside lse
+  kChkPartial = 7,    // split partial row inside the workspace
+  kChkItem = 8,       // work-item fields (head, query tiles, key ranges) inside the tensors
+  kChkSimtRow = 9,    // fp32 path: a row it reads or writes
+  kChkMerge = 10,     // merge: a partial it reads or a row it writes
+};
+#ifdef BAT_DEBUG
+__device__ __forceinline__ bool debug_check(uint32_t* status, bool ok, uint32_t code, long long val) {
+  if (!ok && status) {
+    if (atomicCAS(status + 1, 0u, code) == 0u) atomicExch(status + 2, (uint32_t)val);
+    atomicOr(status, 2u);
+  }
+  return ok;
+}
+#define BAT_DCHECK(status, cond, code, val) ::bat::debug_check((status), (cond), (code), (long long)(val))
+#else
+#define BAT_DCHECK(status, cond, code, val) true
+#endif
+
 // Tensor-core path (bf16 in, fp32 accumulate), d in {64, 128}.
 struct alignas(64) TcParams {
   CUtensorMap tm_q, tm_ks, tm_vs, tm_kc, tm_vc;  // [T, H*d] 2-D maps, box 64 x 128, 128B swizzle
@@ -21,9 +51,12 @@ struct alignas(64) TcParams {
   int32_t T_suf, H;
   float scale_log2;     // softmax scale * log2(e)
   int32_t pad0;
-  uint32_t* status;     // device status word (bit 0: a wait timed out)
+  uint32_t* status;     // device status words (bit 0 of word 0: a wait timed out; debug checks)
   uint64_t wait_ns;     // bound on every spin-wait
   int32_t* item_counter;  // next work item to hand out (zeroed before each launch)
+  int32_t T_cache;      // rows of the cache tensors (bounds checks of debug builds)
+  int32_t n_slots;      // partial slots in the workspace (bounds checks of debug builds)
+  int32_t chk_shrink;   // debug builds: the checks treat every tensor as this many rows shorter
 };
 
 // CUDA-core fp32 path, d in {32, 64, 128}.
@@ -37,6 +70,9 @@ struct SimtParams {
   float* part_lse;
   int32_t T_suf, H;
   float scale;
+  int32_t T_cache, n_slots;
+  uint32_t* status;
+  int32_t chk_shrink;
 };
 
 struct MergeParams {
@@ -47,6 +83,9 @@ struct MergeParams {
   void* out;
   float* lse;
   int32_t T_suf, H;
+  int32_t n_slots;
+  uint32_t* status;
+  int32_t chk_shrink;
 };
 
 constexpr int kPackBatch = 128;
@@ -66,7 +105,8 @@ cudaError_t launch_attn_simt(int d, const SimtParams& p, cudaStream_t s);
 cudaError_t launch_merge(int d, bool out_bf16, const MergeParams& p, cudaStream_t s);
 cudaError_t launch_pack(const void* ks, const void* vs, void* kc, void* vc, const PackBatch& b,
                         int64_t max_bytes, cudaStream_t s);
-// Address of this device's status word (resolved once per device).
+// Address of this device's status words [4] (word 0: status bits; 1, 2: first failed debug
+// check and its value).
 cudaError_t device_status_word(uint32_t** out);
 
 }  // namespace bat

@@ -19,7 +19,10 @@
 //   * the array keeps whatever the last call left.  Nothing needs to start at zero: every
 //     partial slot a split plan reads is written earlier in the same call;
 //   * the first call on each device resolves the array's device address (with that device
-//     current); make that first call before any stream capture begins on the device.
+//     current); make that first call before any stream capture begins on the device.  The
+//     address is kept for the life of the process; cudaDeviceReset unloads the library's device
+//     code, after which the kept address is stale, so this entry point must not be called again
+//     on a device that was reset.
 #include <cuda_runtime.h>
 
 #include <cstdio>

@@ -30,6 +30,8 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
+    # The oracle arm maps none of the repository's shared libraries.
+    assert d["repo_libraries_loaded"] == []
 
 
 def test_reference_arm_other_ranks_exit_quietly():
