@@ -11,16 +11,17 @@
 // The CTA streams the item's key tiles through shared memory with TMA, once each, and both
 // query tiles consume every shared tile:
 //
-//   warp 8       TMA producer: Q tiles, then the K tiles (d = 128) into a K ring, or (d = 64)
-//                the K and V tiles into one ring in the order the MMA issuers consume them:
-//                K0, K1, V0, K2, V1, ... (the K tile of key tile j+1 ahead of the V tile of j)
+//   warp 8       TMA producer: takes the work items; Q tiles and the K tiles (d = 128) into a K
+//                ring, or (d = 64) the K and V tiles into one ring in the order the MMA
+//                issuers consume them: K0, K1, V0, K2, V1, ... (the K tile of key tile j+1
+//                ahead of the V tile of j)
 //   warps 9, 10  MMA issuers (one lane each) of tiles A and B: S = Q.K^T (SS), O += P.V
 //                (d = 128: SS, P read from shared memory; d = 64: TS, P read from TMEM).  S of
 //                key tile j+1 is issued as soon as the softmax has read S of tile j, so it is
 //                computed while the softmax of tile j runs; PV of tile j follows its P (at
 //                d = 64 in two 64-key halves, each as soon as its half of P is written).
-//   warp 11      d = 128: TMA producer of the V tiles into a V ring; d = 64: idle (it
-//                completes the third warpgroup for the register split)
+//   warp 11      d = 128: TMA producer of the V tiles into a V ring; d = 64: TMA producer of
+//                the Q tiles (so the K/V producer streams across item boundaries)
 //   warps 0..3   softmax + epilogue of tile A (one thread per query row = TMEM lane); the
 //                epilogue writes O / l through shared memory with bulk tensor stores
 //   warps 4..7   softmax + epilogue of tile B
@@ -59,7 +60,7 @@ __device__ uint32_t g_status_word[4];
 // (code, clock64) pairs; code = event | x << 8 | index << 16.
 #ifdef BAT_TRACE
 constexpr int kTraceCap = 8192;
-__device__ unsigned long long* g_trace;   // [5 roles][kTraceCap][2]
+__device__ unsigned long long* g_trace;   // [7 roles][kTraceCap][2]
 // The buffer pointer is read once per role (a global load per event would itself stall the
 // traced warp by an L2 round trip).
 __device__ __forceinline__ unsigned long long* trace_base(int role) {
@@ -137,10 +138,12 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// Non-blocking test of an mbarrier phase (test_wait never suspends the thread, unlike
+// try_wait, which may wait for the phase up to a system-dependent limit).
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -330,8 +333,12 @@ struct Cfg {
   static constexpr int kStages = D == 128 ? 3 : 10;
   static constexpr int kStagesK = kTwoRings ? 2 : kStages;
   static constexpr int kStagesV = kStages - kStagesK;
-  // Warps that pop every work item: 8 softmax, 2 MMA issuers and, with two rings, the V producer.
-  static constexpr int kItemConsumers = kTwoRings ? 11 : 10;
+  // Q tiles: loaded by warp 11 when it is not the V producer (d = 64), so the K/V producer never
+  // waits for the next item's Q buffer to free and keeps streaming K/V tiles across item
+  // boundaries; at d = 128 the K producer loads them.
+  static constexpr bool kQWarp = !kTwoRings;
+  // Warps that pop every work item: 8 softmax, 2 MMA issuers and warp 11 (V or Q producer).
+  static constexpr int kItemConsumers = 11;
   // d = 64: PV is issued in two halves of 64 keys, each as soon as the softmax has written that
   // half of P, so the next tile's P can overwrite the first half early (measured faster at
   // d = 64, slower at d = 128, where one PV per tile and one P hand-off are issued instead).
@@ -519,11 +526,15 @@ struct RingGeom {
 // the loads this warp has issued into R.  Returns false on abort.
 template <int D, int R>
 __device__ __forceinline__ bool load_ring(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, const WorkItem& w,
-                                          const Stream& st, uint32_t& ring) {
+                                          const Stream& st, uint32_t& ring, int& trace_n) {
+  (void)trace_n;
   using C = Cfg<D>;
   using G = RingGeom<D, R>;
   const int lane = threadIdx.x & 31;
   const int npos = R == kRingKV ? 2 * st.n : st.n;
+#ifdef BAT_TRACE
+  BAT_TRACE_INIT(R == kRingV ? 6 : 5);   // load events of the K (or shared) ring and of the V ring
+#endif
   for (int pos = 0; pos < npos; ++pos) {
     int j = pos, mask, row0;
     bool is_v = R == kRingV, from_cache;
@@ -542,6 +553,9 @@ __device__ __forceinline__ bool load_ring(const TcParams& p, const Smem<D>& sm, 
       for (int pn = 0; pn < C::kPanels; ++pn)
         tma_load_2d(sm.kv + s * C::kTileBytes + pn * C::kPanelBytes, m, x + pn * 64, y, sm.kv_full + s);
     }
+#ifdef BAT_TRACE
+    BAT_TRACE_EV(0, trace_n, 3, is_v ? 1 : 0, ring);
+#endif
     __syncwarp();
     ++ring;
   }
@@ -562,7 +576,7 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
   const int lane = threadIdx.x & 31;
   uint32_t ring = 0, qcnt[2] = {0, 0}, kq = 0;
   bool ok = true;
-  int tn = 0;
+  int tn = 0, ring_tn = 0;
   (void)tn;
   BAT_TRACE_INIT(0);
   while (ok) {
@@ -595,7 +609,7 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
                  kChkItem, it);
     }
     BAT_TRACE_EV(0, tn, 1, 0, kq);
-    for (int x = 0; ok && x < w.n_q; ++x) {
+    for (int x = 0; ok && !C::kQWarp && x < w.n_q; ++x) {
       ok = wait_bar(sm.q_empty + x, (qcnt[x] & 1) ^ 1, ctl);
       if (!ok) break;
       BAT_TRACE_EV(0, tn, 2, x, kq);
@@ -611,12 +625,48 @@ __device__ void producer_role(const TcParams& p, const Smem<D>& sm, const Ctl& c
       ++qcnt[x];
     }
     const Stream st(w);
-    ok = load_ring<D, C::kTwoRings ? kRingK : kRingKV>(p, sm, ctl, w, st, ring);
+    ok = load_ring<D, C::kTwoRings ? kRingK : kRingKV>(p, sm, ctl, w, st, ring, ring_tn);
   }
   BAT_PHASE_FLUSH();
   if (!ok && lane == 0) {
     // Let every copy this warp issued land before the CTA releases its shared memory.
     drain_ring<D, C::kTwoRings ? kRingK : kRingKV>(sm, ring);
+    for (int x = 0; x < 2; ++x)
+      if (qcnt[x]) drain_bar(sm.q_full + x, (qcnt[x] - 1) & 1);
+  }
+  __syncwarp();
+}
+
+// Q producer (warp 11, d = 64): the query tiles of every item into the two Q buffers, each as
+// soon as the previous item's last S has read that buffer.  It pops the same work items as
+// every other role.
+template <int D>
+__device__ void qproducer_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl) {
+  using C = Cfg<D>;
+  const int lane = threadIdx.x & 31;
+  uint32_t qcnt[2] = {0, 0}, kq = 0;
+  bool ok = true;
+  while (ok) {
+    const int it = pop_item<D>(sm, kq, ctl, ok);
+    if (it < 0) break;
+    const WorkItem w = p.items[it];
+    for (int x = 0; ok && x < w.n_q; ++x) {
+      ok = wait_bar(sm.q_empty + x, (qcnt[x] & 1) ^ 1, ctl);
+      if (!ok) break;
+      if (lane == 0) {
+        int y = x ? w.qB_row0 : w.qA_row0, cx = w.head * D;
+        if (!BAT_DCHECK(p.status, y >= 0 && y < (p.T_suf - p.chk_shrink) && cx >= 0 && cx + D <= p.H * D, kChkQLoad, y))
+          y = cx = 0;
+        mbar_expect_tx(sm.q_full + x, C::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d(sm.q + x * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q, cx + pn * 64, y, sm.q_full + x);
+      }
+      __syncwarp();
+      ++qcnt[x];
+    }
+  }
+  if (!ok && lane == 0) {
     for (int x = 0; x < 2; ++x)
       if (qcnt[x]) drain_bar(sm.q_full + x, (qcnt[x] - 1) & 1);
   }
@@ -630,12 +680,13 @@ __device__ void vproducer_role(const TcParams& p, const Smem<D>& sm, const Ctl& 
   const int lane = threadIdx.x & 31;
   uint32_t ring = 0, kq = 0;
   bool ok = true;
+  int ring_tn = 0;
   while (ok) {
     const int it = pop_item<D>(sm, kq, ctl, ok);
     if (it < 0) break;
     const WorkItem w = p.items[it];
     const Stream st(w);
-    ok = load_ring<D, kRingV>(p, sm, ctl, w, st, ring);
+    ok = load_ring<D, kRingV>(p, sm, ctl, w, st, ring, ring_tn);
   }
   if (!ok && lane == 0) drain_ring<D, kRingV>(sm, ring);
   __syncwarp();
@@ -725,6 +776,9 @@ __device__ void mma_role(const TcParams& p, const Smem<D>& sm, const Ctl& ctl, u
         ph = (r / C::kStages) & 1;
       }
       if (pos == 0) BAT_TRACE_EV(1 + X, tn, 6, X, s_issued);
+#ifdef BAT_TRACE
+      BAT_TRACE_EV(1 + X, tn, 8, is_v ? 1 : 0, C::kTwoRings ? (is_v ? vr0 + j : kr0 + j) : kr0 + pos);
+#endif
       ok = wait_bar(sm.kv_full + s, ph, ctl);
       if (!ok) break;
       if (!mine || !((mask >> X) & 1)) {
@@ -1168,6 +1222,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) bat_attn_tc_kernel(const __grid
     if (warp == 8) producer_role<D>(p, sm, ctl);
     else if (warp == 9 || warp == 10) mma_role<D>(p, sm, ctl, tmem, warp - 9);
     else if constexpr (C::kTwoRings) vproducer_role<D>(p, sm, ctl);
+    else qproducer_role<D>(p, sm, ctl);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
     softmax_role<D>(p, sm, ctl, tmem, warp >> 2);

@@ -9,10 +9,11 @@ issuer has completed), TMA loads complete in any order.  The scheduler runs ever
 role, then completes one random pending operation; if no role can run and nothing is in
 flight, the protocol has deadlocked.  The roles follow the kernel:
 
-  producer     pops work items from the global list into the item queue, loads Q tiles, then
-               the K tiles into the K ring (two rings) or K and V tiles into the shared ring
-               in consumption order K0, K1, V0, K2, V1, ..., V(n-1)
+  producer     pops work items from the global list into the item queue; with two rings it
+               loads the Q tiles, then the K tiles into the K ring; with one ring it loads the
+               K and V tiles into the shared ring in consumption order K0, K1, V0, K2, V1, ...
   vproducer    (two rings) pops the items and loads the V tiles into the V ring
+  qproducer    (one ring) pops the items and loads the Q tiles
   mma X        walks the tiles in consumption order: S of key tile j+1 (K slot landed,
                Q landed for the first S, the softmax has read the previous S), then PV of
                tile j (V slot landed, P written, per P half); frees each slot by a commit or,
@@ -130,7 +131,7 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
     bars = {n: [Bar(f"{n}{x}", c) for x in range(k)] for n, c, k in (
         ("q_full", 1, 2), ("q_empty", 1, 2), ("s_full", 1, 2), ("s_free", 128, 2), ("p_full", 128, 4),
         ("pv_done", 1, 4))}
-    consumers = 2 + 8 + (1 if two_rings else 0)           # MMA issuers, softmax warps, V producer
+    consumers = 2 + 8 + 1                                 # MMA issuers, softmax warps, V or Q producer
     itq_full = [Bar(f"itq_full{i}", 1) for i in range(ITEM_QUEUE)]
     itq_empty = [Bar(f"itq_empty{i}", consumers) for i in range(ITEM_QUEUE)]
     itq = [None] * ITEM_QUEUE
@@ -167,7 +168,7 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
             k += 1
             if w is None:
                 return
-            for x in range(int(w["n_q"])):
+            for x in range(int(w["n_q"]) if two_rings else 0):
                 yield ("wait", bars["q_empty"][x], (qcnt[x] & 1) ^ 1)
                 bars["q_full"][x].expect_tx(1)
                 tma_q.append((bars["q_full"][x], 1))
@@ -193,6 +194,20 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
             for _ in range(Stream(ev[1]).n):
                 yield from load(v_full, v_empty, r)
                 r += 1
+
+    def qproducer():
+        qcnt = [0, 0]
+        for ev in pop(1):
+            if ev[0] != "item":
+                yield ev
+                continue
+            if ev[1] is None:
+                return
+            for x in range(int(ev[1]["n_q"])):
+                yield ("wait", bars["q_empty"][x], (qcnt[x] & 1) ^ 1)
+                bars["q_full"][x].expect_tx(1)
+                tma_q.append((bars["q_full"][x], 1))
+                qcnt[x] += 1
 
     def mma(X):
         q = mma_q[X]
@@ -284,8 +299,7 @@ def simulate(items, two_rings: bool, k_stages: int, v_stages: int, shared_stages
             pv_base += n
 
     roles = {"producer": producer(), "mma0": mma(0), "mma1": mma(1), "softmax0": softmax(0), "softmax1": softmax(1)}
-    if two_rings:
-        roles["vproducer"] = vproducer()
+    roles["vproducer" if two_rings else "qproducer"] = vproducer() if two_rings else qproducer()
     waiting = {k: None for k in roles}
     done = set()
     for _ in range(max_steps):

@@ -64,9 +64,10 @@ for dt, d in (("bf16", 128), ("bf16", 64), ("fp32", 64)):
         out = torch.zeros_like(x["q"])
         bat.bat_attention_forward(plan, x["q"], x["k_suf"], x["v_suf"], x["k_cache"], x["v_cache"], out=out)
         st = bat.bat_get_device_status()
-    print(dt, d, st, bat.last_error())
+        msg = bat.last_error()   # read before the plan's release clears this thread's message
+    print(dt, d, st, msg)
     assert st == bat.BAT_ERR_DEVICE_CHECK, (dt, d, st)
-    assert "bounds check failed" in bat.last_error()
+    assert "bounds check failed" in msg
     assert bat.bat_get_device_status() == bat.BAT_OK   # reported once, then cleared
 print("negative control ok")
 """
