@@ -4,9 +4,11 @@
 
 One step is one pass of the forward over one batch of the named workload (default: the
 mixed bipartite batch, 32768 requests, run as the fewest request-disjoint launches that fit
-in device memory).  Prints one JSON line on rank 0.  Under torchrun each rank serves its own
-batch (weak scaling, rank-seeded inputs, no collective on the data path); the step time is
-the max over ranks of device time measured with CUDA events.
+in device memory).  Prints one JSON line on rank 0.  Under torchrun the one batch is split
+over the ranks by prefix group (hot prefixes replicated, cold ones on the rank that holds
+them, prefixes a rank lacks fetched once from their owner by NCCL send/recv before the timed
+steps; no collective inside a step): strong scaling, the step time is the max over ranks of
+device time measured with CUDA events.
 
 ``--impl reference`` times the fp64 CPU oracle instead (the reference arm): on rank 0 only,
 on a bounded sample of the same workload.
@@ -339,7 +341,7 @@ def run_reference(args, rank, world):
     cores = blas_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload + ("/prefix-side" if args.prefix_side else ""), "sample_requests": n,
                        "requests": tab.R, "H": spec.H, "d": spec.d},
             "requests_per_s": n * args.steps / dt,
@@ -355,6 +357,49 @@ def run_reference(args, rank, world):
 # GPU arm
 
 SECONDARY = ("long-user-history", "item-as-prefix", "user-as-prefix")
+
+
+def shard_batch(full, spec, rank, world, dev):
+    """This rank's share of one batch and its local prefix pool.  The pool starts sharded by
+    prefix id (every rank draws the whole pool from one seed and keeps the prefixes it owns, so
+    a prefix's K/V is the same on every rank); `place` assigns the request groups, and the
+    prefixes a rank needs but does not own are fetched from their owners by NCCL send/recv
+    (timed with CUDA events, max over ranks).  Returns (local table, pool tensors, fetch record)."""
+    import torch
+    import torch.distributed as dist
+    from prefix_shared_attention_b200.sharding import bat_copy_rows, exchange_prefixes, hash_owner, local_table, place
+    owner = hash_owner(full.P, world)
+    pl = place(full.prefix_len, full.req_prefix, full.suffix_len, world, spec.H, spec.d, owner=owner)
+    everything = device_tensors(full, spec.H, spec.d, spec.dtype, spec.seed, device=dev, which=("k_cache", "v_cache"))
+    owned = np.flatnonzero(owner == rank)
+    po = full.prefix_offsets
+    lens = full.prefix_len[owned]
+    dst = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    ok_ = torch.empty((int(dst[-1]), spec.H, spec.d), dtype=everything["k_cache"].dtype, device=dev)
+    ov_ = torch.empty_like(ok_)
+    bat_copy_rows(everything["k_cache"], everything["v_cache"],
+                  [(int(po[p]), int(full.prefix_len[p]), int(dst[i])) for i, p in enumerate(owned) if full.prefix_len[p]],
+                  ok_, ov_)
+    torch.cuda.synchronize()
+    del everything
+    torch.cuda.empty_cache()
+    dist.barrier()   # a collective before the first point-to-point batch, as NCCL requires
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    k_pool, v_pool, nbytes = exchange_prefixes(pl, rank, world, full.prefix_len, owned, ok_, ov_,
+                                               copy_rows=bat_copy_rows)
+    b.record()
+    torch.cuda.synchronize()
+    fetch_ms = max_over_ranks(a.elapsed_time(b), dev)
+    del ok_, ov_
+    torch.cuda.empty_cache()
+    tab, _ = local_table(pl, rank, full)
+    total = torch.tensor([float(nbytes), float(len(pl.fetch[rank]))], dtype=torch.float64, device=dev)
+    dist.all_reduce(total)
+    rec = {"ms": fetch_ms, "bytes": float(total[0].item()), "prefixes": int(total[1].item()),
+           "hot_prefixes": int(len(pl.hot)), "load_imbalance": float(pl.load.max() / pl.load.mean()),
+           "timed": "once before the forward steps (not inside them)"}
+    return tab, {"k_cache": k_pool, "v_cache": v_pool}, rec
 
 
 def roofline_of(flops, nbytes, kernel_s, peaks):
@@ -461,12 +506,21 @@ def main():
     if args.prefix_side:
         from workloads import prefix_side_table
         tab = prefix_side_table(tab)
+    full = tab
+    seed = spec.seed + 1000 * rank
+    fetch = None
+    if world > 1:
+        # The one batch split over the ranks: hot prefixes replicated, cold ones on the rank that
+        # holds them (a pool sharded by prefix id), groups moved off an overloaded owner fetch
+        # their prefix from it (point-to-point copies over NVLink).
+        tab, cache, fetch = shard_batch(full, spec, rank, world, dev)
+    else:
+        cache = device_tensors(tab, spec.H, spec.d, spec.dtype, seed, device=dev, which=("k_cache", "v_cache"))
     free, total = torch.cuda.mem_get_info()
+    # fits_launches budgets the resident pool itself, which is already allocated here.
+    free += sum(t.numel() * t.element_size() for t in cache.values())
     n_launch = args.launches or fits_launches(tab, spec, free, elt)
     parts = split_launches(tab, n_launch)
-    seed = spec.seed + 1000 * rank
-
-    cache = device_tensors(tab, spec.H, spec.d, spec.dtype, seed, device=dev, which=("k_cache", "v_cache"))
     rows = max(p.T_suf for p in parts)
     suf = device_tensors(parts[0], spec.H, spec.d, spec.dtype, seed + 1, device=dev, which=("q", "k_suf", "v_suf"),
                          rows=rows)
@@ -521,8 +575,11 @@ def main():
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     ms_per_step = elapsed_ms / args.steps
-    value = whole_job_rate(step_flops, world, args.steps, elapsed_ms) / 1e12
-    req_s = whole_job_rate(tab.R, world, args.steps, elapsed_ms)
+    # Every rank serves its share of the one batch: the job's rate is the whole batch's work over
+    # the slowest rank's time (strong scaling; at one rank the share is the batch).
+    job_flops = workload_flops_bytes(full, spec.H, spec.d, elt)[0]
+    value = job_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    req_s = full.R * args.steps / (elapsed_ms * 1e-3)
     peaks, peak_kinds = load_peaks()
     achieved = step_flops / (sum(kernel_ms) * 1e-3) / 1e12
     # Which roof binds: algorithmic FLOP per byte against the ridge of the measured peaks.
@@ -624,8 +681,8 @@ def main():
             b_ev.record(s_out)
             torch.cuda.synchronize()
             e_ms = max_over_ranks(a.elapsed_time(b_ev), dev)
-            e2e = {"value": whole_job_rate(step_flops, world, args.e2e_steps, e_ms) / 1e12, "unit": UNIT,
-                   "h2d_bytes_per_step": int(3 * tab.T_suf * row_b), "d2h_bytes_per_step": int(tab.T_suf * row_b),
+            e2e = {"value": job_flops * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+                   "h2d_bytes_per_step": int(3 * full.T_suf * row_b), "d2h_bytes_per_step": int(full.T_suf * row_b),
                    "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
                    "pipeline": f"{len(parts2)} launches over 2 buffer sets; copy-in, forward, copy-out on 3 streams"}
             for pl in plans2:
@@ -642,7 +699,8 @@ def main():
     secondary = None
     if not (args.no_secondary or args.subset or args.prefix_side or args.workload != "mixed"):
         # One launch of each other bf16 workload, on every rank (same steps everywhere).
-        secondary = {name: time_secondary(name, dev, load_peaks()[0]) for name in SECONDARY}
+        if world == 1:
+            secondary = {name: time_secondary(name, dev, load_peaks()[0]) for name in SECONDARY}
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -651,13 +709,14 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload + (f"[:{args.subset}]" if args.subset else "")
                                    + ("/prefix-side" if args.prefix_side else ""), "requests": tab.R, "launches": n_launch, "H": spec.H, "d": spec.d,
                        "prefixes_cached": tab.P, "tokens_suffix": tab.T_suf, "tokens_cache": tab.T_cache,
                        "l2": "inputs larger than L2 (%.0f GB per launch)" % (step_bytes / n_launch / 1e9),
-                       "parallelism": f"dp{world}" if world > 1 else "single"},
+                       "parallelism": (f"{world} ranks, one batch split by prefix group (hot replicated, cold "
+                                       f"sharded)" if world > 1 else "single")},
             "requests_per_s": req_s,
             "plan_ms": plan_ms,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -675,6 +734,8 @@ def main():
         }
         if secondary is not None:
             line["secondary"] = secondary
+        if fetch is not None:
+            line["prefix_fetch"] = fetch
         if hbm_bound:
             # Left of the ridge: the bandwidth roof binds; report against the measured copy rate.
             gbs = step_bytes / (sum(kernel_ms) * 1e-3) / 1e9
