@@ -7,13 +7,16 @@ Python binding never import it, and the oracle imports nothing from them: the
 two share no code.  Inputs for both come from the separate ``workloads``
 generator module.
 
-What it computes is the plain definition of the operation, written out with
+What it computes is the plain definition of each operation, written out with
 no blocking, fusion or reordering beyond what the definition states; see
-``oracle.attention`` for the definition and the readings it rests on.
+``oracle.attention`` (bipartite prefix-shared attention) and ``oracle.gbla``
+(gated bidirectional linear attention) for the definitions and the readings
+they rest on.
 
-Parity status: every function here is pinned by ``tests/test_oracle.py``
-(brute force, closed forms, the four invariants, a library routine); none is
-"parity unpinned".
+Parity status: every function here is pinned, by ``tests/test_oracle.py``
+(brute force, closed forms, the four invariants, a library routine) and by
+``tests/test_gbla_oracle.py`` (element-by-element loops, the linear-time form,
+closed forms, invariants, planted mistakes); none is "parity unpinned".
 """
 
 from .attention import (  # noqa: F401
@@ -25,3 +28,4 @@ from .attention import (  # noqa: F401
     chunk_partial,
     prefix_side_attention,
 )
+from . import gbla  # noqa: F401
