@@ -359,6 +359,55 @@ def run_reference(args, rank, world):
 SECONDARY = ("long-user-history", "item-as-prefix", "user-as-prefix")
 
 
+def gbla_work(seq_lens, H, d=128):
+    """Algorithmic FLOPs and bytes of one GBLA layer: the state (2 T d^2 per head) and the output
+    (2 T d^2 per head) contractions; q, k, v, z and the gate logits read once, y written once."""
+    T = float(sum(seq_lens))
+    return 4.0 * T * d * d * H, (5.0 * T * H * d + T * H) * 2.0
+
+
+def time_gbla(dev, peaks, reps=10, warmup=3):
+    """CUDA-event time of the GBLA layer (state, reduce and output kernels) on the long-history
+    batch, L2 flushed before every timed launch, clocks sampled meanwhile."""
+    import torch
+    import prefix_shared_attention_b200 as bat
+    from workloads import GBLA_LONG_HISTORY as W, gbla_tensors
+    x, so = gbla_tensors(W["seq_lens"], W["H"], W["seed"], device=dev)
+    y = torch.empty_like(x["q"])
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    with bat.GblaPlan(so, W["H"]) as plan:
+        ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+        fwd = lambda: bat.bat_gbla_forward(plan, x["q"], x["k"], x["v"], x["a"], x["z"], x["cq"], x["ck"], x["cv"],
+                                           x["g"], y=y, workspace=ws, stream=stream)
+        for _ in range(warmup):
+            fwd()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        clocks = clock_sampler(dev.index)
+        clocks.start()
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fwd()
+            b.record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        if bat.bat_get_device_status() != bat.BAT_OK:
+            raise RuntimeError(bat.last_error())
+        n_chunks = len(plan.chunks())
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ms[len(ms) // 2]
+    flops, nbytes = gbla_work(W["seq_lens"], W["H"])
+    r = {"workload": W["description"], "ms": med, "tflops": flops / (med * 1e-3) / 1e12,
+         "tokens_per_s": float(sum(W["seq_lens"])) / (med * 1e-3), "launches": 3, "chunks": n_chunks, "reps": reps,
+         "l2": "flushed before every timed launch", "roofline": roofline_of(flops, nbytes, med * 1e-3, peaks),
+         "clocks": clk}
+    del x, y, flush, ws
+    torch.cuda.empty_cache()
+    return r
+
+
 def shard_batch(full, spec, rank, world, dev):
     """This rank's share of one batch and its local prefix pool.  The pool starts sharded by
     prefix id (every rank draws the whole pool from one seed and keeps the prefixes it owns, so
@@ -701,6 +750,8 @@ def main():
         # One launch of each other bf16 workload, on every rank (same steps everywhere).
         if world == 1:
             secondary = {name: time_secondary(name, dev, load_peaks()[0]) for name in SECONDARY}
+            # The second workload: one GBLA layer over long user histories (HBM-bound).
+            secondary["gbla-long-history"] = time_gbla(dev, load_peaks()[0])
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -204,6 +204,67 @@ bat_status bat_attention_forward_noalloc(const bat_plan* plan, const void* q, co
                                          float scale, bat_dtype dt, void* out, float* lse,
                                          void* stream);
 
+/*
+ * Second workload: GBLA, gated bidirectional linear attention ("Gated Bidirectional Linear
+ * Attention for Generative Retrieval", sections "Abstract" and the summary above it): linear-
+ * time attention with no mask over each user history, extended by a local causal convolution
+ * of q, k and v, a per-token key gate that softly forgets tokens, and a gated RMSNorm output.
+ * The page gives no formulas; the library computes, per sequence and head (d = 128):
+ *     x~[t] = sum_{j<4} c_x[j] * x[t-j] (zero before the sequence's first token; x = q, k, v)
+ *     o[t]  = sum_s w[s] phi(q~[t]).phi(k~[s]) v~[s] / (sum_s w[s] phi(q~[t]).phi(k~[s]) + 1e-6)
+ *             with phi(x) = elu(x) + 1 and the key gate w[s] = sigmoid(a[s])
+ *     y[t]  = o[t] / sqrt(mean(o[t]^2) + 1e-6) * g * silu(z[t])
+ * in linear time, through the sequence state S = sum_s w[s] phi(k~[s]) v~[s]^T and n.
+ */
+typedef struct bat_gbla_plan bat_gbla_plan;
+
+/*
+ * bat_gbla_plan_create - work list of one batch of sequences.
+ *   seq_offsets  HOST int64 [n_seqs + 1], non-decreasing: sequence i owns token rows
+ *                [so[i], so[i+1]) of every [T, H, ...] tensor of bat_gbla_forward
+ *   H, d         heads and head width (d must be 128)
+ *   num_sms      SMs to spread the chunks over (0 = the current device's count)
+ *   host_only    1 = build the work list on the host only (inspectable, not runnable)
+ *   out          receives the plan; release it with bat_gbla_plan_destroy
+ * Errors: BAT_ERR_INVALID_ARG (bad offsets, H <= 0, T beyond int32), BAT_ERR_UNSUPPORTED
+ * (d != 128), BAT_ERR_OOM, BAT_ERR_CUDA.
+ */
+bat_status bat_gbla_plan_create(const int64_t* seq_offsets, int32_t n_seqs, int32_t H, int32_t d,
+                                int32_t num_sms, int32_t host_only, void* stream,
+                                bat_gbla_plan** out);
+
+/* Releases the plan (synchronises the device first, through cudaFree).  NULL is accepted. */
+bat_status bat_gbla_plan_destroy(bat_gbla_plan* plan);
+
+/* Device workspace bat_gbla_forward needs: the chunks' partial states and each sequence's
+ * state (about 66 KB per chunk plus 33 KB per sequence and head). */
+size_t bat_gbla_workspace_bytes(const bat_gbla_plan* plan);
+
+/* Copies the work list (32-byte chunk records: pair, head, seq_lo, seq_hi, tile0, n_tiles, 2
+ * pads) into dst (host) when dst is non-NULL and large enough; *n_chunks receives the count.
+ * Diagnostics and tests only. */
+bat_status bat_gbla_plan_chunks(const bat_gbla_plan* plan, void* dst, size_t dst_bytes,
+                                int64_t* n_chunks);
+
+/*
+ * bat_gbla_forward - the GBLA layer for every token of the plan's sequences.
+ *   q, k, v, z      device bf16 [T, H, 128] (z: the output gate)
+ *   a               device bf16 [T, H]: key-gate logits
+ *   conv_q/k/v      device fp32 [H, 4, 128]: depthwise causal convolution taps (tap j
+ *                   multiplies the token j positions back)
+ *   norm_weight     device fp32 [H, 128]
+ *   y               device bf16 [T, H, 128] (written)
+ *   workspace       device scratch of at least bat_gbla_workspace_bytes(plan) bytes
+ * All device pointers 16-byte aligned (a: 2-byte).  Asynchronous on `stream`; three kernel
+ * launches (state, reduce, output).  One plan and workspace run on one stream at a time.
+ * Errors: BAT_ERR_INVALID_ARG (null or misaligned pointer, workspace too small, host-only
+ * plan, wrong device), BAT_ERR_CUDA.
+ */
+bat_status bat_gbla_forward(const bat_gbla_plan* plan, const void* q, const void* k, const void* v,
+                            const void* a, const void* z, const float* conv_q, const float* conv_k,
+                            const float* conv_v, const float* norm_weight, void* y, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reports and clears the device-side status word of the
  * current device: BAT_ERR_DEVICE_CHECK if a bounds check of a debug build failed (the message
  * names the check and the offending value), BAT_ERR_TIMEOUT if a kernel abandoned a bounded

@@ -19,6 +19,7 @@ _BINDING_NAMES = (
     "BAT_ERR_UNSUPPORTED", "LIB_PATH", "MERGE_JOB_DTYPE", "WORK_ITEM_DTYPE", "BatError", "Plan",
     "bat_attention_forward", "bat_attention_forward_noalloc", "bat_get_device_status", "bat_prefix_kv_build",
     "bat_set_wait_timeout_ns", "bat_version", "bat_debug_checks", "BAT_ERR_DEVICE_CHECK", "exported_symbols", "last_error", "prefix_build",
+    "GblaPlan", "GBLA_CHUNK_DTYPE", "bat_gbla_forward",
 )
 
 __all__ = list(_BINDING_NAMES) + ["algorithmic_bytes", "algorithmic_flops"]

@@ -69,6 +69,11 @@ _SIGNATURES = {
     "bat_last_error": (C.c_char_p, []),
     "bat_version": (_i32, []),
     "bat_debug_checks": (_i32, []),
+    "bat_gbla_plan_create": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, C.POINTER(_vp)]),
+    "bat_gbla_plan_destroy": (_i32, [_vp]),
+    "bat_gbla_workspace_bytes": (_sz, [_vp]),
+    "bat_gbla_plan_chunks": (_i32, [_vp, _vp, _sz, C.POINTER(_i64)]),
+    "bat_gbla_forward": (_i32, [_vp] + [_vp] * 10 + [_vp, _sz, _vp]),
 }
 
 
@@ -202,6 +207,70 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+GBLA_CHUNK_DTYPE = np.dtype([(n, np.int32) for n in ("pair", "head", "seq_lo", "seq_hi", "tile0", "n_tiles",
+                                                      "pad0", "pad1")])
+
+
+class GblaPlan:
+    """Owns a ``bat_gbla_plan``: the chunk list of one batch of sequences for the GBLA layer."""
+
+    def __init__(self, seq_offsets, H: int, d: int = 128, num_sms: int = 0, host_only: bool = False, stream=None):
+        self._so = np.ascontiguousarray(seq_offsets, dtype=np.int64)
+        n = int(self._so.shape[0]) - 1
+        if n < 0:
+            raise BatError(BAT_ERR_INVALID_ARG, "seq_offsets needs at least one entry")
+        h = C.c_void_p()
+        st = None if host_only else _stream_handle(stream)
+        check(lib.bat_gbla_plan_create(_ptr(self._so), n, H, d, num_sms, 1 if host_only else 0, st, C.byref(h)))
+        self.handle = h
+        self.H, self.d = H, d
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(lib.bat_gbla_workspace_bytes(self.handle))
+
+    def chunks(self) -> np.ndarray:
+        n = C.c_int64()
+        check(lib.bat_gbla_plan_chunks(self.handle, None, 0, C.byref(n)))
+        out = np.zeros(n.value, dtype=GBLA_CHUNK_DTYPE)
+        check(lib.bat_gbla_plan_chunks(self.handle, _ptr(out), out.nbytes, C.byref(n)))
+        return out
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            check(lib.bat_gbla_plan_destroy(self.handle))
+        self.handle = C.c_void_p()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def bat_gbla_forward(plan: GblaPlan, q, k, v, a, z, conv_q, conv_k, conv_v, norm_weight, y=None, workspace=None,
+                     stream=None):
+    """GBLA layer on torch device tensors (q, k, v, z bf16 [T, H, 128]; a bf16 [T, H]; conv_* fp32
+    [H, 4, 128]; norm_weight fp32 [H, 128]); allocates ``y`` and the workspace when not given.
+    Returns ``y``."""
+    import torch
+    if y is None:
+        y = torch.empty_like(q)
+    need = plan.workspace_bytes
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ptrs = [t.data_ptr() for t in (q, k, v, a, z, conv_q, conv_k, conv_v, norm_weight, y)]
+    check(lib.bat_gbla_forward(plan.handle, *ptrs, workspace.data_ptr(), int(workspace.numel()),
+                               _stream_handle(stream)))
+    return y
 
 
 def bat_prefix_kv_build(k_src, v_src, src_offsets, dst_offsets, k_cache, v_cache, stream=None) -> None:

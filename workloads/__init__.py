@@ -44,6 +44,8 @@ __all__ = [
     "host_tensors",
     "device_tensors",
     "zipf_ranks",
+    "GBLA_LONG_HISTORY",
+    "gbla_tensors",
 ]
 
 
@@ -294,3 +296,27 @@ def gather_requests(table: RequestTable, tensors: dict, reqs, out=None):
     if out is not None:
         host["out"] = take(out, rows)
     return sub, host, rows
+
+
+# GBLA (gated bidirectional linear attention, the second workload): a batch of long user
+# histories.  The GBLA page quotes its single-layer speed at a history length of 32768; the
+# batch and head count are this build's choice (8 histories, 8 heads of width 128).
+GBLA_LONG_HISTORY = {"name": "gbla-long-history", "seq_lens": [32768] * 8, "H": 8, "d": 128, "seed": 5,
+                     "description": "8 user histories x 32768 tokens, H=8, d=128, bf16 (q, k, v, z N(0,1); "
+                                    "gate logits N(0, 2^2); conv taps N(0, 0.6^2); norm weight 1 + N(0, 0.2^2))"}
+
+
+def gbla_tensors(seq_lens, H: int, seed: int, device="cpu", d: int = 128):
+    """Seeded inputs of the GBLA layer: q, k, v, z bf16 [T, H, d] ~ N(0,1); key-gate logits a bf16
+    [T, H] ~ N(0, 2^2); causal-convolution taps cq, ck, cv fp32 [H, 4, d] ~ N(0, 0.6^2); norm weight
+    g fp32 [H, d] ~ 1 + N(0, 0.2^2).  Returns (dict, seq_offsets)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    T = int(sum(seq_lens))
+    rn = lambda *shape: torch.randn(*shape, generator=g, device=device)
+    x = {"q": rn(T, H, d).bfloat16(), "k": rn(T, H, d).bfloat16(), "v": rn(T, H, d).bfloat16(),
+         "z": rn(T, H, d).bfloat16(), "a": (2.0 * rn(T, H)).bfloat16(),
+         "cq": 0.6 * rn(H, 4, d), "ck": 0.6 * rn(H, 4, d), "cv": 0.6 * rn(H, 4, d), "g": 1.0 + 0.2 * rn(H, d)}
+    so = np.concatenate([[0], np.cumsum(np.asarray(seq_lens, np.int64))]).astype(np.int64)
+    return x, so
