@@ -1,9 +1,13 @@
 // C ABI of the GBLA path (declared in include/bat.h): the work list of a batch of user
 // histories, argument checks and the kernel launches.  No arithmetic of the layer happens
 // here; it all runs in bat_gbla.cu's kernels.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -44,6 +48,32 @@ constexpr int64_t kPartFloats = 128 * 128 + 128;
 
 int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D map over a bf16 [T, H*128] tensor: box 64 columns x box_rows rows; zero fill outside it.
+bool encode(CUtensorMap* m, const void* base, int64_t T, int32_t H, uint32_t box_rows, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)H * 128, (cuuint64_t)(T > 0 ? T : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)H * 128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -78,16 +108,43 @@ bat_status bat_gbla_plan_create(const int64_t* seq_offsets, int32_t n_seqs, int3
   plan->H = H;
   plan->d = d;
   plan->T = T;
-  // Chunks: about two per SM (two CTAs fit per SM), each a run of consecutive tiles of one
-  // (sequence, head), the tiles of a pair split as evenly as possible.
+  // Chunks: runs of consecutive tiles of one (sequence, head), one CTA each, one CTA per SM.
+  // Their count is a whole number of waves over the SMs (about 24 tiles per chunk), dealt to the
+  // pairs in proportion to their tiles (largest remainder), so every CTA gets about the same
+  // number of tiles.
+  std::vector<int32_t> tiles_of;
   int64_t total_tiles = 0;
-  for (int32_t i = 0; i < n_seqs; ++i) total_tiles += H * ((seq_offsets[i + 1] - seq_offsets[i] + 127) / 128);
-  const int64_t per_chunk = std::max<int64_t>(1, (total_tiles + 2 * num_sms - 1) / (2 * num_sms));
   for (int32_t i = 0; i < n_seqs; ++i) {
-    const int64_t L = seq_offsets[i + 1] - seq_offsets[i];
-    const int32_t tiles = (int32_t)((L + 127) / 128);
+    const int32_t tiles = (int32_t)((seq_offsets[i + 1] - seq_offsets[i] + 127) / 128);
+    tiles_of.push_back(tiles);
+    total_tiles += (int64_t)H * tiles;
+  }
+  const int64_t waves = std::max<int64_t>(1, (int64_t)std::llround((double)total_tiles / (num_sms * 24.0)));
+  const int64_t target = num_sms * waves;
+  std::vector<int32_t> nc_of(n_seqs, 0);
+  {
+    std::vector<std::pair<double, int32_t>> frac;
+    int64_t given = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+      if (tiles_of[i] == 0) continue;
+      const double share = total_tiles ? (double)target * tiles_of[i] / (double)total_tiles : 0.0;   // per head
+      nc_of[i] = (int32_t)std::min<double>(tiles_of[i], std::max(1.0, std::floor(share)));
+      given += (int64_t)H * nc_of[i];
+      frac.push_back({share - std::floor(share), i});
+    }
+    std::sort(frac.begin(), frac.end(), [](const auto& a, const auto& b) { return a.first > b.first; });
+    for (const auto& f : frac) {
+      if (given + H > target) break;
+      if (nc_of[f.second] < tiles_of[f.second]) {
+        ++nc_of[f.second];
+        given += H;
+      }
+    }
+  }
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const int32_t tiles = tiles_of[i];
     if (tiles == 0) continue;
-    const int32_t nc = (int32_t)((tiles + per_chunk - 1) / per_chunk);
+    const int32_t nc = nc_of[i];
     for (int32_t h = 0; h < H; ++h) {
       bat::GblaPair pr;
       pr.chunk0 = (int32_t)plan->chunks.size();
@@ -187,6 +244,10 @@ bat_status bat_gbla_forward(const bat_gbla_plan* plan, const void* q, const void
   const int64_t nc = (int64_t)plan->chunks.size(), np = (int64_t)plan->pairs.size();
   bat::GblaParams p;
   memset(&p, 0, sizeof(p));
+  if (!encode(&p.tm_q, q, plan->T, plan->H, 136, false) || !encode(&p.tm_k, k, plan->T, plan->H, 136, false) ||
+      !encode(&p.tm_v, v, plan->T, plan->H, 136, false) || !encode(&p.tm_z, z, plan->T, plan->H, 128, true) ||
+      !encode(&p.tm_y, y, plan->T, plan->H, 32, true))
+    return gfail(BAT_ERR_CUDA, "cuTensorMapEncodeTiled failed for a GBLA tensor");
   p.chunks = plan->d_chunks;
   p.pairs = plan->d_pairs;
   p.q = q;

@@ -2,6 +2,7 @@
 // of the three kernels and their parameter block.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -27,7 +28,11 @@ struct GblaPair {
   int32_t chunk0, n_chunks;
 };
 
-struct GblaParams {
+struct alignas(64) GblaParams {
+  // 2-D tensor maps over [T, H * 128] bf16: q, k, v with a box of 64 columns x 136 rows (a tile
+  // and the 8 rows before it) and no swizzle (the threads read them); z with a box of 64 x 128
+  // and y (bulk stores) with 64 x 32, both with the 128-byte swizzle.
+  CUtensorMap tm_q, tm_k, tm_v, tm_z, tm_y;
   const GblaChunk* chunks;
   const GblaPair* pairs;
   const void *q, *k, *v;    // bf16 [T, H, 128]
