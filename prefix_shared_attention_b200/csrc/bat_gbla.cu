@@ -74,8 +74,10 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
 // The same chunk of row `r` of a raw tile (two unswizzled 136-row panels).
 __device__ __forceinline__ uint32_t raw_off(int r, int c) { return (uint32_t)((c >> 3) * kRawPanel + r * 128 + (c & 7) * 16); }
 
-__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : __expf(x); }
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
+// elu(x) + 1, the exponential on the MUFU (2^(x log2 e)).
+__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : ex2(x * 1.4426950408889634f); }
+// sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation.
+__device__ __forceinline__ float sigmoidf_(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -156,6 +158,7 @@ __device__ __forceinline__ void conv_tile(uint32_t raw, const float* w, int c, i
     wt[j][0] = w0.x, wt[j][1] = w0.y, wt[j][2] = w0.z, wt[j][3] = w0.w;
     wt[j][4] = w1.x, wt[j][5] = w1.y, wt[j][6] = w1.z, wt[j][7] = w1.w;
   }
+  // Channel pairs go through the packed fp32x2 FMA.
 #pragma unroll
   for (int i = 0; i < kRows; ++i)
 #pragma unroll
@@ -170,7 +173,7 @@ __device__ __forceinline__ void conv_tile(uint32_t raw, const float* w, int c, i
       const int i = m - 3 + j;
       if (i >= 0 && i < kRows) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) out[i][e] = fmaf(wt[j][e], f[e], out[i][e]);
+        for (int e = 0; e < 8; e += 2) ffma2v(out[i][e], out[i][e + 1], wt[j][e], wt[j][e + 1], f[e], f[e + 1]);
       }
     }
   }
@@ -265,22 +268,29 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
     constexpr uint32_t idesc = make_idesc(128, 128, true, true);
     bool ok = true;
     int done = 0;
+    // Gate logits of this thread's rows, loaded one tile ahead (they come from global memory).
+    auto load_gates = [&](int tile, __nv_bfloat16 (&a)[kRows]) {
+      const int64_t tb = (int64_t)lo + (int64_t)(ch.tile0 + tile) * 128 + kRows * g;
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) a[r] = (tile < ch.n_tiles && tb + r < hi) ? ax[(tb + r) * H + h] : __float2bfloat16(0.f);
+    };
+    __nv_bfloat16 a_next[kRows];
+    load_gates(0, a_next);
     for (int i = 0; i < ch.n_tiles; ++i) {
       const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
       const int s = i & 1;
       const uint32_t raw = smem_u32(ring + s * kStateStage);
       float gate[kRows];
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const int64_t t = t0 + kRows * g + r;
-        gate[r] = t < hi ? sigmoidf_(__bfloat162float(ax[t * H + h])) : 0.f;
-      }
+      for (int r = 0; r < kRows; ++r) gate[r] = t0 + kRows * g + r < hi ? sigmoidf_(__bfloat162float(a_next[r])) : 0.f;
+      load_gates(i + 1, a_next);
       ok = wait_phase(&sm.raw_full[s], (i >> 1) & 1, sm, p.status);
+      // The previous tile's MMAs must have read the operand tiles before they are rewritten.
+      if (ok && i > 0) ok = wait_phase(&sm.mma_done, (i - 1) & 1, sm, p.status);
       if (!consumer_all(ok)) {
         ok = false;
         break;
       }
-      uint4 ku[kRows], vu[kRows];
       {
         float x[kRows][8];
         conv_tile(raw, sm.w[0], c, g, t0, lo, x);
@@ -288,9 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
         for (int r = 0; r < kRows; ++r) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[r][e] = gate[r] * phi(x[r][e]);
-          ku[r] = pack8(x[r]);
+          const uint4 u = pack8(x[r]);
+          st_shared_v4(smem_u32(A) + sw_off(kRows * g + r, c), u.x, u.y, u.z, u.w);
           float kb[8];
-          unpack8(ku[r], kb);   // n sums exactly the bf16 values the tensor core multiplies
+          unpack8(u, kb);   // n sums exactly the bf16 values the tensor core multiplies
 #pragma unroll
           for (int e = 0; e < 8; ++e) nacc[e] += kb[e];
         }
@@ -299,21 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
         float x[kRows][8];
         conv_tile(raw + 2 * kRawPanel, sm.w[1], c, g, t0, lo, x);
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) vu[r] = pack8(x[r]);
+        for (int r = 0; r < kRows; ++r) {
+          const uint4 u = pack8(x[r]);
+          st_shared_v4(smem_u32(B) + sw_off(kRows * g + r, c), u.x, u.y, u.z, u.w);
+        }
       }
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&sm.raw_empty[s]);   // this warp is done with the raw tile
-      // The previous tile's MMAs must have read the operand tiles before they are rewritten.
-      if (i > 0) ok = wait_phase(&sm.mma_done, (i - 1) & 1, sm, p.status);
-      if (!consumer_all(ok)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        st_shared_v4(smem_u32(A) + sw_off(kRows * g + r, c), ku[r].x, ku[r].y, ku[r].z, ku[r].w);
-        st_shared_v4(smem_u32(B) + sw_off(kRows * g + r, c), vu[r].x, vu[r].y, vu[r].z, vu[r].w);
-      }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       consumer_sync();
       if (warp == 0) {
@@ -529,10 +532,13 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         const uint32_t za = zt + sw_off(r, chunk);
         float zf[8], yv[8];
         unpack8(ld_shared_v4(za), zf);
+        const float4 g0 = *reinterpret_cast<const float4*>(gw + 8 * chunk);
+        const float4 g1 = *reinterpret_cast<const float4*>(gw + 8 * chunk + 4);
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float zz = zf[e];
-          yv[e] = __uint_as_float(v[8 * k4 + e]) * scale * gw[8 * chunk + e] * (zz / (1.f + __expf(-zz)));
+          yv[e] = __uint_as_float(v[8 * k4 + e]) * scale * gg[e] * (zz * sigmoidf_(zz));   // silu(z)
         }
         const uint4 yu = pack8(yv);
         if (whole) st_shared_v4(za, yu.x, yu.y, yu.z, yu.w);
