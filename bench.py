@@ -93,15 +93,29 @@ def workload_flops_bytes(tab, H, d, elt):
             algorithmic_bytes(tab.prefix_len, tab.req_prefix, tab.suffix_len, H, d, elt))
 
 
-def traffic_per_launch(workload, kernel_src):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this exact
-    kernel source; else None."""
+KERNEL_SOURCES = ("bat_attn_tc.cu", "bat_ptx.h", "bat_kernels.h")
+
+
+def kernel_source_hash():
+    """First 16 hex digits of the SHA-256 of the attention kernel's sources, in a fixed order."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_launch(workload, alg_bytes_per_launch):
+    """DRAM bytes per launch from the committed ncu summary of this workload, if it was taken on
+    the current kernel sources; else None.  A capture of a smaller launch of the same workload
+    (the first requests and the prefixes they read) is scaled to this launch by algorithmic
+    bytes: the ratio of measured to algorithmic traffic is what the capture measures."""
     path = os.path.join(ROOT, "profiles", f"bat_attn_tc_{workload}_traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path))
-    h = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
-    return rec.get("dram_bytes_per_launch") if rec.get("kernel_sha256_16") == h else None
+    if rec.get("kernel_sha256_16") != kernel_source_hash():
+        return None
+    return rec["dram_bytes_per_launch"] / rec["alg_bytes_per_launch"] * alg_bytes_per_launch
 
 
 class NvmlClockSampler:
@@ -366,12 +380,18 @@ def gbla_work(seq_lens, H, d=128):
     return 4.0 * T * d * d * H, (5.0 * T * H * d + T * H) * 2.0
 
 
-def time_gbla(dev, peaks, reps=10, warmup=3):
+def time_gbla(dev, peaks, reps=10, warmup=3, n_seqs=0):
     """CUDA-event time of the GBLA layer (state, reduce and output kernels) on the long-history
-    batch, L2 flushed before every timed launch, clocks sampled meanwhile."""
+    batch (or its first `n_seqs` histories), L2 flushed before every timed launch, clocks
+    sampled meanwhile."""
     import torch
     import prefix_shared_attention_b200 as bat
-    from workloads import GBLA_LONG_HISTORY as W, gbla_tensors
+    from workloads import GBLA_LONG_HISTORY
+    from workloads import gbla_tensors
+    W = dict(GBLA_LONG_HISTORY)
+    if n_seqs:
+        W["seq_lens"] = W["seq_lens"][:n_seqs]
+        W["description"] = f"first {n_seqs} of: " + W["description"]
     x, so = gbla_tensors(W["seq_lens"], W["H"], W["seed"], device=dev)
     y = torch.empty_like(x["q"])
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -526,6 +546,9 @@ def main():
                     help="profiling aid: only the first N requests (and the prefixes they read); not a bench line")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the one-launch timings of the other bf16 workloads")
+    ap.add_argument("--gbla", type=int, default=-1, metavar="N_SEQS",
+                    help="profiling aid: time only the GBLA layer on the long-history batch (0: all of its "
+                         "histories, else the first N) and print its record; not a bench line")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference" or os.environ.get("BAT_BENCH_ALLOW_SHORT"), \
         "at least 3 warm-up steps"
@@ -545,6 +568,12 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    if args.gbla >= 0:
+        if rank == 0:
+            rec = time_gbla(dev, load_peaks()[0], reps=max(args.steps, 1), warmup=args.warmup, n_seqs=args.gbla)
+            print(json.dumps(rec), flush=True)
+        return 0
 
     spec = CONFIGS[args.workload]
     assert spec.dtype == "bf16", "the bench times the bf16 tensor-core path"
@@ -638,8 +667,7 @@ def main():
     # against (>= 60 % of it); the sustained figure (the same GEMM back to back for seconds,
     # under the power cap) is reported beside it.
     peak = float(peaks["bf16_tflops"])
-    kernel_src = os.path.join(ROOT, "prefix_shared_attention_b200", "csrc", "bat_attn_tc.cu")
-    traffic = None if args.prefix_side else traffic_per_launch(args.workload, kernel_src)
+    traffic = None if (args.prefix_side or args.subset) else traffic_per_launch(args.workload, step_bytes / n_launch)
 
     # End to end through the public API with host buffers: every launch's request tokens (q,
     # k, v) go host -> device from pinned memory, the forward runs, the output comes back.  The

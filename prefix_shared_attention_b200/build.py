@@ -1,6 +1,6 @@
 """Build libbat.so in-tree for sm_100a.
 
-    python -m prefix_shared_attention_b200.build [--force] [--verbose] [--debug]
+    python -m prefix_shared_attention_b200.build [--force] [--verbose] [--debug | --phase]
 
 Every CUDA source is compiled with nvcc for ``sm_100a`` only (tcgen05, TMA) and linked
 with the static CUDA runtime into ``prefix_shared_attention_b200/libbat.so``.  Objects go
@@ -11,6 +11,10 @@ rebuild of their object.
 ``-DBAT_DEBUG``: its kernels check every tensor-map coordinate and store index against the
 tensors' bounds and report a failed check through the device status word (no check traps).
 Select it at run time with ``BAT_LIBRARY=<path to libbat_debug.so>``.
+
+``--phase`` builds ``libbat_phase.so`` (objects in ``_build_phase/``), compiled with
+``-DBAT_PHASE``: every warp of the attention kernel adds up the clocks it spends in each phase
+of its loop and writes the totals once at its end (``phase_profile.py`` runs and reports it).
 """
 
 from __future__ import annotations
@@ -30,6 +34,8 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libbat.so")
 BUILD_DEBUG = os.path.join(PKG, "_build_debug")
 LIB_DEBUG = os.path.join(PKG, "libbat_debug.so")
+BUILD_PHASE = os.path.join(PKG, "_build_phase")
+LIB_PHASE = os.path.join(PKG, "libbat_phase.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-I", INCLUDE, "-I", CSRC,
@@ -56,9 +62,11 @@ def _mtime(p):
     return os.path.getmtime(p) if os.path.exists(p) else -1.0
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
-    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
-    flags = FLAGS + (["-DBAT_DEBUG"] if debug else [])
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False,
+          phase: bool = False) -> str:
+    assert not (debug and phase), "one variant at a time"
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD_PHASE, LIB_PHASE) if phase else (BUILD, LIB)
+    flags = FLAGS + (["-DBAT_DEBUG"] if debug else []) + (["-DBAT_PHASE"] if phase else [])
     os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     newest_header = max(_mtime(h) for h in headers())
@@ -98,8 +106,9 @@ def main():
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
     ap.add_argument("--debug", action="store_true", help="build libbat_debug.so (device-side bounds checks)")
+    ap.add_argument("--phase", action="store_true", help="build libbat_phase.so (per-warp phase clocks)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_verbose, a.debug))
+    print(build(a.force, a.verbose, a.ptxas_verbose, a.debug, a.phase))
 
 
 if __name__ == "__main__":
