@@ -12,18 +12,22 @@
 //
 // Three kernels; the two that stream the tokens are pipelined alike.  One CTA per SM: a
 // producer warp loads 128-token tiles (plus the 8 rows before them, for the convolution) into
-// a two-stage ring with TMA; eight consumer warps read them from shared memory, apply the
+// two-stage rings with TMA; sixteen consumer warps read them from shared memory (each thread 8
+// consecutive rows x 4 channels, so the convolution reads 11 raw rows per 8 outputs), apply the
 // convolution, feature map and gate in fp32 registers, write bf16 operand tiles in the 128-byte-
 // swizzled layout, and one elected thread issues the tile's tcgen05.mma.  The next tiles' loads
 // are in flight while a tile is computed.
 //   gbla_state_kernel   per chunk (consecutive tiles of one (sequence, head)):
-//                       D[d x d] += (w phi(k~))^T v~ (M = d, N = d, K = tokens; both operands
-//                       MN-major); the partial state and n go to the workspace.
+//                       D[d x (d+16)] += (w phi(k~))^T [v~ | 1] (M = d, N = d + 16, K = tokens;
+//                       both operands MN-major; the ones column gives n); the partial state and
+//                       n go to the workspace.
 //   gbla_reduce_kernel  sums the chunks' partials of each (sequence, head) into S (bf16) and n.
-//   gbla_out_kernel     per chunk: S into shared memory once; per tile phi(q~) (K-major) and
-//                       O = phi(q~) . S into TMEM; the epilogue (one thread per token row) divides
-//                       by n . phi(q~), normalises and gates with z (loaded by TMA beside q), writes
-//                       y over z in shared memory and stores it with bulk tensor stores.
+//   gbla_out_kernel     per chunk: [S | n] into shared memory once; per tile phi(q~) (K-major)
+//                       and [O | n . phi(q~)] = phi(q~) . [S | n] into one of two TMEM
+//                       accumulators; the epilogue of the previous tile (four warps per row
+//                       quarter, 32 columns each) divides by the denominator, normalises and
+//                       gates with z (its own ring), writes y over z in shared memory and stores
+//                       it with bulk tensor stores.
 // The path is HBM-bound (about 0.4 d FLOP per byte): q, k, v, z and the gate logits are read
 // once and y is written once; S and the partials stay small and in L2.
 #include <cuda.h>
@@ -43,42 +47,61 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumers + 32;     // plus the producer warp (warp 16)
 constexpr int kProducerWarp = kConsumerWarps;
-constexpr int kRows = 128 / (kConsumers / 16);   // rows of a tile per consumer thread (16 threads per row)
+// Consumer thread (warp w, lane l): rows 8w .. 8w+7 of a tile, channels 4l .. 4l+3.
+constexpr int kRowsT = 8;
 constexpr int kPanel = 128 * 128;             // one 64-column panel of a 128-row bf16 tile
 constexpr int kRawRows = 136;                 // a tile's 128 rows plus the 8 before them
 constexpr int kRawPanel = kRawRows * 128;     // one 64-column panel of a raw (unswizzled) tile
 constexpr int kStateStage = 4 * kRawPanel;    // raw k and v
-constexpr int kOutStage = 2 * kRawPanel + 2 * kPanel;   // raw q, then z (128-byte swizzled)
+constexpr int kQStage = 2 * kRawPanel;        // raw q
+constexpr int kZStage = 2 * kPanel;           // z (128-byte swizzled), then y over it
+// MMA width: the 128 channels plus a third operand panel whose first column carries a ones
+// column (state: n = (w phi(k~))^T 1) or n itself (output: n . phi(q~)), so the tensor core
+// produces n and the denominator beside the product.
+constexpr int kN = 144;
+constexpr uint32_t kAccStride = 256;          // TMEM columns between the output kernel's two accumulators
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kEpsAttn = 1e-6f;
 constexpr float kEpsNorm = 1e-6f;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 struct GblaSmem {
-  float w[2][4 * 128];   // convolution taps (state: k, v; output: q)
-  float vec[3][128];     // state: n partial; output: n, norm weight
-  float den[2][128];     // output: n . phi(q~) of the tile, double-buffered
-  float ss[4][128];      // output: partial sums of squares of each row, per 32-column block
-  uint64_t raw_full[2], raw_empty[2], mma_done;
+  float w[2][4 * 128];              // convolution taps (state: k, v; output: q)
+  float gw[128];                    // output: norm weight
+  float ss[4][128];                 // output: partial sums of squares of each row, per 32-column block
+  uint64_t full[2][2], empty[2][2];   // [ring][stage]
+  uint64_t mma_done[2];             // per accumulator (the state kernel uses one)
   uint32_t tmem_slot;
   int abort;
 };
-constexpr size_t kStateSmem = 1024 + 4 * kPanel + 2 * kStateStage + sizeof(GblaSmem);
-constexpr size_t kOutSmem = 1024 + 4 * kPanel + 2 * kOutStage + sizeof(GblaSmem);
+constexpr size_t kStateSmem = 1024 + 5 * kPanel + 2 * kStateStage + sizeof(GblaSmem);
+constexpr size_t kOutSmem = 1024 + 5 * kPanel + 2 * kQStage + 2 * kZStage + sizeof(GblaSmem);
 static_assert(kStateSmem <= 227 * 1024 && kOutSmem <= 227 * 1024, "shared memory budget");
 
-// 16-byte chunk `c` (8 elements, c in 0..15) of row `r` of a 128-row bf16 tile held as two
-// 64-column panels with the 128-byte swizzle (chunk index XOR row mod 8).
+// Byte offset of 8-byte piece c4 (4 elements, c4 in 0..31) of row r of a 128-row bf16 tile held
+// as two 64-column panels with the 128-byte swizzle (16-byte chunk index XOR row mod 8).
+__device__ __forceinline__ uint32_t sw_off8(int r, int c4) {
+  return (uint32_t)((c4 >> 4) * kPanel + r * 128 + ((((c4 >> 1) & 7) ^ (r & 7)) << 4) + ((c4 & 1) << 3));
+}
+// 16-byte chunk c (8 elements, c in 0..15) of row r of the same layout.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return (uint32_t)((c >> 3) * kPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
-// The same chunk of row `r` of a raw tile (two unswizzled 136-row panels).
-__device__ __forceinline__ uint32_t raw_off(int r, int c) { return (uint32_t)((c >> 3) * kRawPanel + r * 128 + (c & 7) * 16); }
+// The same 8-byte piece of row r of a raw tile (two unswizzled 136-row panels).
+__device__ __forceinline__ uint32_t raw_off8(int r, int c4) {
+  return (uint32_t)((c4 >> 4) * kRawPanel + r * 128 + (c4 & 15) * 8);
+}
 
-// elu(x) + 1, the exponential on the MUFU (2^(x log2 e)).
-__device__ __forceinline__ float phi(float x) { return x > 0.f ? x + 1.f : ex2(x * 1.4426950408889634f); }
+// elu(x) + 1 = exp(min(x, 0)) + max(x, 0): no branch, one MUFU operation.
+__device__ __forceinline__ float phi(float x) { return ex2(fminf(x, 0.f) * kLog2e) + fmaxf(x, 0.f); }
 // sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation.
 __device__ __forceinline__ float sigmoidf_(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
+__device__ __forceinline__ void unpack4(const uint2& u, float (&f)[4]) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  f[0] = a.x, f[1] = a.y, f[2] = b.x, f[3] = b.y;
+}
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -88,7 +111,9 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     f[2 * i + 1] = t.y;
   }
 }
-
+__device__ __forceinline__ uint2 pack4(const float (&v)[4]) {
+  return make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
 __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
   uint4 u;
   u.x = pack_bf16x2(v[0], v[1]);
@@ -98,10 +123,28 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
   return u;
 }
 
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+  uint2 u;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(u.x), "=r"(u.y) : "r"(addr));
+  return u;
+}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 u;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
   return u;
+}
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, const uint2& u) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(u.x), "r"(u.y) : "memory");
+}
+
+// One TMEM column of this warp's 32 lanes.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\ttcgen05.wait::ld.sync.aligned;"
+               : "=r"(r)
+               : "r"(taddr)
+               : "memory");
+  return __uint_as_float(r);
 }
 
 // Barrier of the consumer warps (the producer warp does not take part).
@@ -116,6 +159,8 @@ __device__ __forceinline__ bool consumer_all(bool ok) {
       : "memory");
   return r != 0;
 }
+// Barrier of the four consumer warps that read TMEM lane quarter qd (warps qd, qd+4, qd+8, qd+12).
+__device__ __forceinline__ void quarter_sync(int qd) { asm volatile("bar.sync %0, 128;" ::"r"(2 + qd) : "memory"); }
 
 // Bounded wait on an mbarrier phase; false on timeout or when the CTA is aborting.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, GblaSmem& sm, uint32_t* status) {
@@ -139,83 +184,113 @@ __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity) {
     if (global_ns() - t0 > kWaitNs / 10) break;
 }
 
-// This thread's kRows rows (kRows*g .. of the tile) and 8 channels (16-byte chunk c) after the
-// causal convolution of width 4, from a raw tile in shared memory whose row 8 is the tile's
-// first token; rows before the sequence start count as zero.
-__device__ __forceinline__ void conv_tile(uint32_t raw, const float* w, int c, int g, int64_t t0, int lo,
-                                          float (&out)[kRows][8]) {
-  uint4 r[kRows + 3];
+// The causal convolution (width 4) of this thread's 8 rows (8g .. 8g+7 of the tile) and 4
+// channels (piece c4) from a raw tile in shared memory whose row 8 is the tile's first token;
+// tokens before the sequence start count as zero.  The 11 raw rows stream through once; output
+// row i is handed to emit(i, x) as soon as its last tap has been added, so at most four rows of
+// sums are live.
+template <class Emit>
+__device__ __forceinline__ void conv8(uint32_t raw, const float* taps, int c4, int g, int64_t t0, int lo, Emit&& emit) {
+  float4 w[4];
 #pragma unroll
-  for (int i = 0; i < kRows + 3; ++i) {
-    const int row = kRows * g + 5 + i;   // token t0 + kRows*g - 3 + i
-    r[i] = (t0 + kRows * g - 3 + i >= lo) ? ld_shared_v4(raw + raw_off(row, c)) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  float wt[4][8];
+  for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(taps + j * 128 + 4 * c4);
+  float acc[kRowsT][4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float4 w0 = *reinterpret_cast<const float4*>(w + j * 128 + c * 8);
-    const float4 w1 = *reinterpret_cast<const float4*>(w + j * 128 + c * 8 + 4);
-    wt[j][0] = w0.x, wt[j][1] = w0.y, wt[j][2] = w0.z, wt[j][3] = w0.w;
-    wt[j][4] = w1.x, wt[j][5] = w1.y, wt[j][6] = w1.z, wt[j][7] = w1.w;
-  }
-  // Channel pairs go through the packed fp32x2 FMA.
+  for (int i = 0; i < kRowsT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 #pragma unroll
-  for (int i = 0; i < kRows; ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) out[i][e] = 0.f;
-#pragma unroll
-  for (int m = 0; m < kRows + 3; ++m) {
-    float f[8];
-    unpack8(r[m], f);
-    // Raw row m feeds output rows i = m - 3 + j for taps j = 0..3.
+  for (int m = 0; m < kRowsT + 3; ++m) {
+    // Raw row m is token t0 + 8g - 3 + m; it meets tap j in output row i = m - 3 + j.
+    uint2 u = make_uint2(0u, 0u);
+    if (t0 + kRowsT * g - 3 + m >= lo) u = ld_shared_v2(raw + raw_off8(kRowsT * g + 5 + m, c4));
+    float f[4];
+    unpack4(u, f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = m - 3 + j;
-      if (i >= 0 && i < kRows) {
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) ffma2v(out[i][e], out[i][e + 1], wt[j][e], wt[j][e + 1], f[e], f[e + 1]);
+      if (i >= 0 && i < kRowsT) {
+        ffma2v(acc[i][0], acc[i][1], w[j].x, w[j].y, f[0], f[1]);
+        ffma2v(acc[i][2], acc[i][3], w[j].z, w[j].w, f[2], f[3]);
       }
     }
+    if (m >= 3) emit(m - 3, acc[m - 3]);
   }
 }
 
-__device__ __forceinline__ void tmem_alloc128(uint32_t* slot) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(128u)
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(cols)
                : "memory");
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void tmem_free128(uint32_t tmem) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128u) : "memory");
+__device__ __forceinline__ void tmem_free(uint32_t tmem, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols) : "memory");
 }
 
-// Producer warp: the chunk's tiles into the two-stage ring.  Map m's two 64-column panels go
-// to offset map_off[m] of the stage, starting `rows_before[m]` rows before the tile (8 for the
-// raw tiles the convolution reads, 0 for z); drains its loads if the CTA aborts.
-template <int kStage>
-__device__ __forceinline__ void produce(const GblaChunk& ch, GblaSmem& sm, uint8_t* ring, const CUtensorMap* const* maps,
-                                        const int* rows_before, const int* map_off, int nmaps, uint32_t* status) {
+// A two-stage ring of tiles filled by the producer warp: `nmaps` tensors per stage, each as two
+// 64-column panels of `panel` bytes starting `before` rows before the tile.
+struct Ring {
+  const CUtensorMap* map[2];
+  int nmaps, before, panel, stage;
+  uint8_t* base;
+  uint64_t *full, *empty;
+};
+
+// Producer warp: tile i of the chunk into stage i % 2 of every ring, in ring order; drains its
+// loads if the CTA aborts.
+__device__ __forceinline__ void produce(const GblaChunk& ch, GblaSmem& sm, const Ring* rings, int nrings,
+                                        uint32_t* status) {
   const int lane = threadIdx.x & 31;
-  int issued = 0;
-  for (int i = 0; i < ch.n_tiles; ++i) {
+  int issued[2] = {0, 0};
+  bool ok = true;
+  for (int i = 0; ok && i < ch.n_tiles; ++i) {
     const int s = i & 1;
-    if (!wait_phase(&sm.raw_empty[s], ((i >> 1) & 1) ^ 1, sm, status)) break;
-    if (lane == 0) {
-      const int y0 = ch.seq_lo + (ch.tile0 + i) * 128;
-      mbar_expect_tx(&sm.raw_full[s], kStage);
-      for (int m = 0; m < nmaps; ++m)
+    for (int q = 0; q < nrings; ++q) {
+      const Ring& R = rings[q];
+      if (!wait_phase(&R.empty[s], ((i >> 1) & 1) ^ 1, sm, status)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        const int y0 = ch.seq_lo + (ch.tile0 + i) * 128;
+        mbar_expect_tx(&R.full[s], R.stage);
+        for (int m = 0; m < R.nmaps; ++m)
 #pragma unroll
-        for (int pn = 0; pn < 2; ++pn)
-          tma_load_2d(ring + s * kStage + map_off[m] + pn * (rows_before[m] ? kRawPanel : kPanel), maps[m],
-                      ch.head * 128 + pn * 64, y0 - rows_before[m], &sm.raw_full[s]);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_2d(R.base + s * R.stage + (2 * m + pn) * R.panel, R.map[m], ch.head * 128 + pn * 64, y0 - R.before,
+                        &R.full[s]);
+      }
+      __syncwarp();
+      ++issued[q];
     }
-    __syncwarp();
-    ++issued;
   }
-  if (issued < ch.n_tiles && lane == 0) {
+  if (!ok && lane == 0) {
     // Aborting: let the loads in flight land before the CTA releases its shared memory.
-    for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) drain_phase(&sm.raw_full[i & 1], (i >> 1) & 1);
+    for (int q = 0; q < nrings; ++q)
+      for (int i = (issued[q] > 2 ? issued[q] - 2 : 0); i < issued[q]; ++i)
+        drain_phase(&rings[q].full[i & 1], (i >> 1) & 1);
   }
   __syncwarp();
+}
+
+__device__ __forceinline__ void init_barriers(GblaSmem& sm, int nrings) {
+  for (int q = 0; q < nrings; ++q)
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.full[q][s], 1);
+      mbar_init(&sm.empty[q][s], kConsumerWarps);   // one arrival per consumer warp
+    }
+  mbar_init(&sm.mma_done[0], 1);
+  mbar_init(&sm.mma_done[1], 1);
+  sm.abort = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Row r of the third (64-column) panel of a 128-row operand tile: value x in its first column,
+// zeros elsewhere.
+__device__ __forceinline__ void write_extra_row(uint8_t* panel, int r, float x) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t v0 = k == 0 ? pack_bf16x2(x, 0.f) : 0u;
+    st_shared_v4(smem_u32(panel) + r * 128 + ((k ^ (r & 7)) << 4), v0, 0u, 0u, 0u);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -225,98 +300,80 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
   extern __shared__ uint8_t dyn[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* A = base;                // (w phi(k~)) tile: rows = tokens, columns = d (MN-major A)
-  uint8_t* B = base + 2 * kPanel;   // v~ tile: rows = tokens, columns = d (MN-major B)
-  uint8_t* ring = base + 4 * kPanel;
+  uint8_t* B = base + 2 * kPanel;   // [v~ | 1] tile: rows = tokens, columns = d + 16 (MN-major B)
+  uint8_t* ring = base + 5 * kPanel;
   GblaSmem& sm = *reinterpret_cast<GblaSmem*>(ring + 2 * kStateStage);
   const GblaChunk ch = p.chunks[blockIdx.x];
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int c = tid & 15, g = (tid >> 4) & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
-  if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], kConsumerWarps);   // one arrival per consumer warp
-    }
-    mbar_init(&sm.mma_done, 1);
-    sm.abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
+  if (tid == 0) init_barriers(sm, 1);
   for (int i = tid; i < 4 * 128; i += kThreads) {
     sm.w[0][i] = p.conv_k[h * 4 * 128 + i];
     sm.w[1][i] = p.conv_v[h * 4 * 128 + i];
   }
-  if (tid < 128) sm.vec[0][tid] = 0.f;
-  if (warp == 0) tmem_alloc128(&sm.tmem_slot);
-  if (warp == kProducerWarp && (tid & 31) == 0) {
+  // The ones column: n = sum over tokens of w phi(k~) comes out of the MMA as column d.
+  if (tid < 128) write_extra_row(B + 2 * kPanel, tid, 1.f);
+  if (warp == 0) tmem_alloc(&sm.tmem_slot, 256);
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
 
   if (warp == kProducerWarp) {
-    const CUtensorMap* maps[2] = {&p.tm_k, &p.tm_v};
-    const int before[2] = {8, 8}, off[2] = {0, 2 * kRawPanel};
-    produce<kStateStage>(ch, sm, ring, maps, before, off, 2, p.status);
+    const Ring r0 = {{&p.tm_k, &p.tm_v}, 2, 8, kRawPanel, kStateStage, ring, sm.full[0], sm.empty[0]};
+    produce(ch, sm, &r0, 1, p.status);
   } else {
-    float nacc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) nacc[e] = 0.f;
+    const int g = warp, c4 = lane;
     const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
-    constexpr uint32_t idesc = make_idesc(128, 128, true, true);
+    constexpr uint32_t idesc = make_idesc(128, kN, true, true);
     bool ok = true;
     int done = 0;
-    // Gate logits of this thread's rows, loaded one tile ahead (they come from global memory).
-    auto load_gates = [&](int tile, __nv_bfloat16 (&a)[kRows]) {
-      const int64_t tb = (int64_t)lo + (int64_t)(ch.tile0 + tile) * 128 + kRows * g;
+    // Gate logits of this warp's rows (the same for every lane), loaded one tile ahead.
+    auto load_gates = [&](int tile, __nv_bfloat16 (&a)[kRowsT]) {
+      const int64_t tb = (int64_t)lo + (int64_t)(ch.tile0 + tile) * 128 + kRowsT * g;
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) a[r] = (tile < ch.n_tiles && tb + r < hi) ? ax[(tb + r) * H + h] : __float2bfloat16(0.f);
+      for (int r = 0; r < kRowsT; ++r)
+        a[r] = (tile < ch.n_tiles && tb + r < hi) ? ax[(tb + r) * H + h] : __float2bfloat16(0.f);
     };
-    __nv_bfloat16 a_next[kRows];
+    __nv_bfloat16 a_next[kRowsT];
     load_gates(0, a_next);
     for (int i = 0; i < ch.n_tiles; ++i) {
       const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
       const int s = i & 1;
       const uint32_t raw = smem_u32(ring + s * kStateStage);
-      float gate[kRows];
+      float gate[kRowsT];
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) gate[r] = t0 + kRows * g + r < hi ? sigmoidf_(__bfloat162float(a_next[r])) : 0.f;
+      for (int r = 0; r < kRowsT; ++r)
+        gate[r] = t0 + kRowsT * g + r < hi ? sigmoidf_(__bfloat162float(a_next[r])) : 0.f;
       load_gates(i + 1, a_next);
-      ok = wait_phase(&sm.raw_full[s], (i >> 1) & 1, sm, p.status);
-      // The previous tile's MMAs must have read the operand tiles before they are rewritten.
-      if (ok && i > 0) ok = wait_phase(&sm.mma_done, (i - 1) & 1, sm, p.status);
+      ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      // Both operand tiles are computed into registers first, then stored once the previous
+      // tile's MMAs have read the operand buffers.
+      uint2 uk[kRowsT], uv[kRowsT];
+      conv8(raw, sm.w[0], c4, g, t0, lo, [&](int r, float (&x)[4]) {
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[e] = gate[r] * phi(x[e]);
+        uk[r] = pack4(y);
+      });
+      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, t0, lo, [&](int r, float (&x)[4]) { uv[r] = pack4(x); });
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[0][s]);   // this warp is done with the raw tile
+      if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
       if (!consumer_all(ok)) {
         ok = false;
         break;
       }
-      {
-        float x[kRows][8];
-        conv_tile(raw, sm.w[0], c, g, t0, lo, x);
 #pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[r][e] = gate[r] * phi(x[r][e]);
-          const uint4 u = pack8(x[r]);
-          st_shared_v4(smem_u32(A) + sw_off(kRows * g + r, c), u.x, u.y, u.z, u.w);
-          float kb[8];
-          unpack8(u, kb);   // n sums exactly the bf16 values the tensor core multiplies
-#pragma unroll
-          for (int e = 0; e < 8; ++e) nacc[e] += kb[e];
-        }
+      for (int r = 0; r < kRowsT; ++r) {
+        st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
+        st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), uv[r]);
       }
-      {
-        float x[kRows][8];
-        conv_tile(raw + 2 * kRawPanel, sm.w[1], c, g, t0, lo, x);
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          const uint4 u = pack8(x[r]);
-          st_shared_v4(smem_u32(B) + sw_off(kRows * g + r, c), u.x, u.y, u.z, u.w);
-        }
-      }
-      __syncwarp();
-      if ((tid & 31) == 0) mbar_arrive(&sm.raw_empty[s]);   // this warp is done with the raw tile
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       consumer_sync();
       if (warp == 0) {
@@ -326,39 +383,40 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
         for (int kk = 0; kk < 8; ++kk)   // 16 tokens per step: two 8-row swizzle groups (2 KiB)
           mma_ss_w(tmem, ad + (uint64_t)(kk * 2048 / 16), bd + (uint64_t)(kk * 2048 / 16), idesc,
                    (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit_w(&sm.mma_done);
+        tc_commit_w(&sm.mma_done[0]);
       }
       done = i + 1;
     }
-    // Partial n: this thread's 8 channels summed over its rows, then over the 16 row groups.
-#pragma unroll
-    for (int e = 0; e < 8; ++e) atomicAdd(&sm.vec[0][c * 8 + e], nacc[e]);
     if (done > 0) {
-      if (ok) ok = wait_phase(&sm.mma_done, (done - 1) & 1, sm, p.status);
-      else drain_phase(&sm.mma_done, (done - 1) & 1);
+      if (ok) ok = wait_phase(&sm.mma_done[0], (done - 1) & 1, sm, p.status);
+      else drain_phase(&sm.mma_done[0], (done - 1) & 1);
     }
     ok = consumer_all(ok);
     tc_fence_after();
     float* part = p.part_s + (int64_t)blockIdx.x * (128 * 128 + 128);
     {
       // Row i = 32 * (warp % 4) + lane of the partial state (channel i of phi(k~)), columns
-      // 32 * (warp / 4) .. +31 (v channels): one 32-column TMEM load per warp.
+      // 32 * (warp / 4) .. +31 (v channels): one 32-column TMEM load per warp; column d is n.
       const int qd = warp & 3, cb = warp >> 2;
-      const int i = 32 * qd + (tid & 31);
+      const int i = 32 * qd + lane;
+      const bool keep = ok && done > 0;
       float4* dst = reinterpret_cast<float4*>(part + (int64_t)i * 128 + 32 * cb);
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * cb, r);
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        dst[e] = (ok && done > 0) ? make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                                __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-      if (tid < 128) part[128 * 128 + tid] = sm.vec[0][tid];
+        dst[e] = keep ? make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                                    __uint_as_float(r[4 * e + 3]))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (cb == 0) {
+        const float nv = tmem_ld1(tmem + ((uint32_t)(32 * qd) << 16) + 128);
+        part[128 * 128 + i] = keep ? nv : 0.f;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_free128(tmem);
+  if (warp == 0) tmem_free(tmem, 256);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -378,51 +436,41 @@ __global__ void __launch_bounds__(256) gbla_reduce_kernel(const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------------------
-// Output: y for every token of one chunk.
+// Output: y for every token of one chunk.  The MMA of tile i runs while the epilogue of tile
+// i - 1 reads the other TMEM accumulator; q and z come through separate rings because z is
+// needed one tile later than q.
 
 __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_constant__ GblaParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* A = base;                 // phi(q~) tile: rows = tokens, columns = d (K-major A)
-  uint8_t* Bs = base + 2 * kPanel;   // S: rows = phi channels (K), columns = v channels (MN-major B)
-  uint8_t* ring = base + 4 * kPanel;
-  GblaSmem& sm = *reinterpret_cast<GblaSmem*>(ring + 2 * kOutStage);
-  float* nvec = sm.vec[0];
-  float* gw = sm.vec[1];
+  uint8_t* Bs = base + 2 * kPanel;   // [S | n]: rows = phi channels (K), columns = v channels + n (MN-major B)
+  uint8_t* qring = base + 5 * kPanel;
+  uint8_t* zring = qring + 2 * kQStage;
+  GblaSmem& sm = *reinterpret_cast<GblaSmem*>(zring + 2 * kZStage);
   const GblaChunk ch = p.chunks[blockIdx.x];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = tid & 15, g = (tid >> 4) & 31;
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
-  if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], kConsumerWarps);
-    }
-    mbar_init(&sm.mma_done, 1);
-    sm.abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) tmem_alloc128(&sm.tmem_slot);
+  if (tid == 0) init_barriers(sm, 2);
+  if (warp == 0) tmem_alloc(&sm.tmem_slot, 512);
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&p.tm_q);
     prefetch_tmap(&p.tm_z);
     prefetch_tmap(&p.tm_y);
   }
   if (warp < kConsumerWarps) {
-    // S of this (sequence, head) into the B tile (row i, 16-byte chunk c of its 128 columns).
-    const uint4* src = reinterpret_cast<const uint4*>(p.state + (int64_t)ch.pair * 128 * 128);
+    // S of this (sequence, head) into the B tile: rows 8w .. 8w+7, 8-byte piece `lane`.
+    const uint2* src = reinterpret_cast<const uint2*>(p.state + (int64_t)ch.pair * 128 * 128);
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      const int row = kRows * g + r;
-      const uint4 u = src[row * 16 + c];
-      st_shared_v4(smem_u32(Bs) + sw_off(row, c), u.x, u.y, u.z, u.w);
+    for (int r = 0; r < kRowsT; ++r) {
+      const int row = kRowsT * warp + r;
+      st_shared_v2(smem_u32(Bs) + sw_off8(row, lane), src[row * 32 + lane]);
     }
   }
+  // n as the first column of the third panel: the MMA's column d is n . phi(q~).
+  if (tid < 128) write_extra_row(Bs + 2 * kPanel, tid, p.norm_n[(int64_t)ch.pair * 128 + tid]);
   for (int i = tid; i < 4 * 128; i += kThreads) sm.w[0][i] = p.conv_q[h * 4 * 128 + i];
-  if (tid < 128) {
-    nvec[tid] = p.norm_n[(int64_t)ch.pair * 128 + tid];
-    gw[tid] = p.norm_w[h * 128 + tid];
-  }
+  if (tid < 128) sm.gw[tid] = p.norm_w[h * 128 + tid];
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
@@ -430,101 +478,47 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
   const uint32_t tmem = sm.tmem_slot;
 
   if (warp == kProducerWarp) {
-    const CUtensorMap* maps[2] = {&p.tm_q, &p.tm_z};
-    const int before[2] = {8, 0}, off[2] = {0, 2 * kRawPanel};
-    produce<kOutStage>(ch, sm, ring, maps, before, off, 2, p.status);
+    const Ring rings[2] = {{{&p.tm_q, nullptr}, 1, 8, kRawPanel, kQStage, qring, sm.full[0], sm.empty[0]},
+                           {{&p.tm_z, nullptr}, 1, 0, kPanel, kZStage, zring, sm.full[1], sm.empty[1]}};
+    produce(ch, sm, rings, 2, p.status);
   } else {
-    float nv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) nv[e] = nvec[c * 8 + e];
+    const int g = warp, c4 = lane;
     __nv_bfloat16* yx = reinterpret_cast<__nv_bfloat16*>(p.y);
-    constexpr uint32_t idesc = make_idesc(128, 128, true);
+    constexpr uint32_t idesc = make_idesc(128, kN, true);
     // Epilogue roles: warp w reads the TMEM rows of its lane quarter qd = w % 4 (rows 32 qd ..
     // 32 qd + 31) and the 32 columns of block cb = w / 4.
     const int qd = warp & 3, cb = warp >> 2;
     const int r = 32 * qd + lane;
     bool ok = true, stores_pending = false;
     int done = 0;
-    for (int i = 0; i < ch.n_tiles; ++i) {
-      const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
-      const int s = i & 1;
-      const uint32_t stage = smem_u32(ring + s * kOutStage);
-      float* den = sm.den[s];
-      ok = wait_phase(&sm.raw_full[s], (i >> 1) & 1, sm, p.status);
-      if (!consumer_all(ok)) {
-        ok = false;
-        break;
-      }
-      uint4 qu[kRows];
-      {
-        float x[kRows][8];
-        conv_tile(stage, sm.w[0], c, g, t0, lo, x);
-#pragma unroll
-        for (int rr = 0; rr < kRows; ++rr) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[rr][e] = phi(x[rr][e]);
-          qu[rr] = pack8(x[rr]);
-          float fb[8];
-          unpack8(qu[rr], fb);   // the denominator uses exactly the bf16 values the tensor core reads
-          float dsum = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) dsum += fb[e] * nv[e];
-          // Sum over the 16 threads (lanes c = 0..15 of this half-warp) holding the row's chunks.
-#pragma unroll
-          for (int off = 8; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
-          if (c == 0) den[kRows * g + rr] = dsum;
-        }
-      }
-      // The previous tile's MMAs must have read A before it is rewritten.
-      if (i > 0) ok = wait_phase(&sm.mma_done, (i - 1) & 1, sm, p.status);
-      if (!consumer_all(ok)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int rr = 0; rr < kRows; ++rr)
-        st_shared_v4(smem_u32(A) + sw_off(kRows * g + rr, c), qu[rr].x, qu[rr].y, qu[rr].z, qu[rr].w);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      consumer_sync();
-      if (warp == 0) {
-        tc_fence_after();
-        const uint64_t ad = sdesc_sw128(smem_u32(A), 16, 1024), bd = sdesc_sw128(smem_u32(Bs), kPanel, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // 16 channels per step
-          const uint64_t aoff = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
-          mma_ss_w(tmem, ad + aoff, bd + (uint64_t)(kk * 2048 / 16), idesc, kk > 0 ? 1u : 0u);
-        }
-        tc_commit_w(&sm.mma_done);
-      }
-      done = i + 1;
-      // Epilogue, spread over every consumer warp: each row's sum of squares from its four
-      // 32-column blocks, then y = o / den / rms * g * silu(z) for this warp's block, written over
-      // z in the stage (rows of a quarter that lies entirely inside the sequence) or straight to
-      // y with 16-byte stores (a quarter that reaches past the sequence end).
-      ok = wait_phase(&sm.mma_done, i & 1, sm, p.status);
-      if (!consumer_all(ok)) {
-        ok = false;
-        break;
-      }
+
+    // Epilogue of tile j: y = o / den / rms * g * silu(z), written over z in its stage (row
+    // quarters that lie entirely inside the sequence, then bulk tensor stores) or straight to
+    // y with 16-byte stores (a quarter that reaches past the sequence end).
+    auto epilogue = [&](int j) {
+      const int zs = j & 1;
+      const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + j) * 128;
+      const bool zok = wait_phase(&sm.full[1][zs], (j >> 1) & 1, sm, p.status);
       tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(j & 1) * kAccStride + ((uint32_t)(32 * qd) << 16);
       const int64_t t = t0 + r;
-      const bool live = t < hi;
-      const bool whole = t0 + 32 * qd + 31 < hi;
+      const bool live = zok && t < hi;
+      const bool whole = zok && t0 + 32 * qd + 31 < hi;
       uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * cb, v);
-      const float inv_den = 1.f / (den[r] + kEpsAttn);
+      tmem_ld32(acc + 32 * cb, v);
+      const float inv_den = 1.f / (tmem_ld1(acc + 128) + kEpsAttn);
+      tc_fence_before();
       float ssp = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float o = __uint_as_float(v[e]) * inv_den;
-        ssp += o * o;
+        ssp = fmaf(o, o, ssp);
       }
       sm.ss[cb][r] = ssp;
-      tc_fence_before();
-      consumer_sync();
+      quarter_sync(qd);
       const float ss = sm.ss[0][r] + sm.ss[1][r] + sm.ss[2][r] + sm.ss[3][r];
       const float scale = inv_den * rsqrtf(ss * (1.f / 128.f) + kEpsNorm);
-      const uint32_t zt = stage + 2 * kRawPanel;   // z tile: two 128-byte-swizzled panels
+      const uint32_t zt = smem_u32(zring + zs * kZStage);
       uint4* yrow = reinterpret_cast<uint4*>(yx + (live ? (t * H + h) * 128 : 0));
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
@@ -532,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         const uint32_t za = zt + sw_off(r, chunk);
         float zf[8], yv[8];
         unpack8(ld_shared_v4(za), zf);
-        const float4 g0 = *reinterpret_cast<const float4*>(gw + 8 * chunk);
-        const float4 g1 = *reinterpret_cast<const float4*>(gw + 8 * chunk + 4);
+        const float4 g0 = *reinterpret_cast<const float4*>(sm.gw + 8 * chunk);
+        const float4 g1 = *reinterpret_cast<const float4*>(sm.gw + 8 * chunk + 4);
         const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -545,28 +539,67 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         else if (live) yrow[chunk] = yu;
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      consumer_sync();
-      // Warps 0..7, lane 0: one bulk tensor store per (row quarter, 64-column panel) of a quarter
-      // inside the sequence; the stage is released once the stores have read it.
-      if (warp < 8 && lane == 0) {
-        const int sq = warp & 3, pn = warp >> 2;
-        if (t0 + 32 * sq + 31 < hi) {
-          tma_store_2d(&p.tm_y, ring + s * kOutStage + 2 * kRawPanel + pn * kPanel + 32 * sq * 128, h * 128 + pn * 64,
-                       (int)(t0 + 32 * sq));
-          bulk_commit();
-          bulk_wait_read();
-          stores_pending = true;
-        }
+      quarter_sync(qd);
+      // Warps of column blocks 0 and 2, lane 0: one bulk tensor store of this quarter's rows per
+      // 64-column panel; the stage is released once the stores have read it.
+      if ((cb & 1) == 0 && lane == 0 && whole) {
+        const int pn = cb >> 1;
+        tma_store_2d(&p.tm_y, zring + zs * kZStage + pn * kPanel + 32 * qd * 128, h * 128 + pn * 64, (int)(t0 + 32 * qd));
+        bulk_commit();
+        bulk_wait_read();
+        stores_pending = true;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.raw_empty[s]);
+      if (lane == 0) mbar_arrive(&sm.empty[1][zs]);
+    };
+
+    for (int i = 0; i < ch.n_tiles; ++i) {
+      const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
+      const int s = i & 1;
+      ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      uint2 uq[kRowsT];
+      conv8(smem_u32(qring + s * kQStage), sm.w[0], c4, g, t0, lo, [&](int rr, float (&x)[4]) {
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) y[e] = phi(x[e]);
+        uq[rr] = pack4(y);
+      });
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[0][s]);
+      // The previous tile's MMAs must have read A (and finished its accumulator) first.
+      if (ok && i > 0) ok = wait_phase(&sm.mma_done[(i - 1) & 1], ((i - 1) >> 1) & 1, sm, p.status);
+      if (!consumer_all(ok)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int rr = 0; rr < kRowsT; ++rr) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + rr, c4), uq[rr]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      consumer_sync();
+      if (warp == 0) {
+        tc_fence_after();
+        const uint64_t ad = sdesc_sw128(smem_u32(A), 16, 1024), bd = sdesc_sw128(smem_u32(Bs), kPanel, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {   // 16 channels per step
+          const uint64_t aoff = (uint64_t)(((kk >> 2) * kPanel + (kk & 3) * 32) >> 4);
+          mma_ss_w(tmem + (uint32_t)s * kAccStride, ad + aoff, bd + (uint64_t)(kk * 2048 / 16), idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit_w(&sm.mma_done[s]);
+      }
+      if (i > 0) epilogue(i - 1);
+      done = i + 1;
     }
-    if (done > 0 && !ok) drain_phase(&sm.mma_done, (done - 1) & 1);
+    if (done > 0) {
+      const int j = done - 1;
+      if (ok) ok = wait_phase(&sm.mma_done[j & 1], (j >> 1) & 1, sm, p.status);
+      else drain_phase(&sm.mma_done[j & 1], (j >> 1) & 1);
+      if (consumer_all(ok)) epilogue(j);
+    }
     if (stores_pending) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_free128(tmem);
+  if (warp == 0) tmem_free(tmem, 512);
 }
 
 }  // namespace
