@@ -92,8 +92,25 @@ __device__ __forceinline__ uint32_t raw_off8(int r, int c4) {
   return (uint32_t)((c4 >> 4) * kRawPanel + r * 128 + (c4 & 15) * 8);
 }
 
-// elu(x) + 1 = exp(min(x, 0)) + max(x, 0): no branch, one MUFU operation.
-__device__ __forceinline__ float phi(float x) { return ex2(fminf(x, 0.f) * kLog2e) + fmaxf(x, 0.f); }
+// elu(x) + 1 = exp(min(x, 0)) + max(x, 0): no branch, one MUFU operation per element; two
+// elements at a time on the packed fp32x2 path.
+__device__ __forceinline__ void phi2(float& x0, float& x1) {
+  float e0, e1;
+  fmul2v(e0, e1, fminf(x0, 0.f), fminf(x1, 0.f), kLog2e, kLog2e);
+  e0 = ex2(e0);
+  e1 = ex2(e1);
+  fadd2(e0, e1, fmaxf(x0, 0.f), fmaxf(x1, 0.f));
+  x0 = e0, x1 = e1;
+}
+// w * (elu(x) + 1) = 2^(min(x, 0) log2 e + log2 w) + w max(x, 0), the gate w folded into the
+// exponent (lw = log2 w; w = 0 gives lw = -inf and 0).
+__device__ __forceinline__ void gated_phi2(float& x0, float& x1, float w, float lw) {
+  float e0, e1;
+  ffma2c(e0, e1, fminf(x0, 0.f), fminf(x1, 0.f), kLog2e, kLog2e, lw, lw);
+  e0 = ex2(e0);
+  e1 = ex2(e1);
+  ffma2c(x0, x1, fmaxf(x0, 0.f), fmaxf(x1, 0.f), w, w, e0, e1);
+}
 // sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation.
 __device__ __forceinline__ float sigmoidf_(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
@@ -189,27 +206,33 @@ __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity) {
 // tokens before the sequence start count as zero.  The 11 raw rows stream through once; output
 // row i is handed to emit(i, x) as soon as its last tap has been added, so at most four rows of
 // sums are live.
+// `first` = the index of the first raw row at or after the sequence start (<= 0: all of them).
 template <class Emit>
-__device__ __forceinline__ void conv8(uint32_t raw, const float* taps, int c4, int g, int64_t t0, int lo, Emit&& emit) {
+__device__ __forceinline__ void conv8(uint32_t raw, const float* taps, int c4, int g, int first, Emit&& emit) {
   float4 w[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(taps + j * 128 + 4 * c4);
   float acc[kRowsT][4];
-#pragma unroll
-  for (int i = 0; i < kRowsT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  const uint32_t src = raw + raw_off8(kRowsT * g + 5, c4);
 #pragma unroll
   for (int m = 0; m < kRowsT + 3; ++m) {
-    // Raw row m is token t0 + 8g - 3 + m; it meets tap j in output row i = m - 3 + j.
+    // Raw row m is token t0 + 8g - 3 + m; it meets tap j in output row i = m - 3 + j (the
+    // output row's first contribution, tap 3, by a multiply).
     uint2 u = make_uint2(0u, 0u);
-    if (t0 + kRowsT * g - 3 + m >= lo) u = ld_shared_v2(raw + raw_off8(kRowsT * g + 5 + m, c4));
+    if (m >= first) u = ld_shared_v2(src + m * 128);
     float f[4];
     unpack4(u, f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = m - 3 + j;
       if (i >= 0 && i < kRowsT) {
-        ffma2v(acc[i][0], acc[i][1], w[j].x, w[j].y, f[0], f[1]);
-        ffma2v(acc[i][2], acc[i][3], w[j].z, w[j].w, f[2], f[3]);
+        if (j == 3) {
+          fmul2v(acc[i][0], acc[i][1], w[j].x, w[j].y, f[0], f[1]);
+          fmul2v(acc[i][2], acc[i][3], w[j].z, w[j].w, f[2], f[3]);
+        } else {
+          ffma2v(acc[i][0], acc[i][1], w[j].x, w[j].y, f[0], f[1]);
+          ffma2v(acc[i][2], acc[i][3], w[j].z, w[j].w, f[2], f[3]);
+        }
       }
     }
     if (m >= 3) emit(m - 3, acc[m - 3]);
@@ -333,35 +356,39 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
     constexpr uint32_t idesc = make_idesc(128, kN, true, true);
     bool ok = true;
     int done = 0;
-    // Gate logits of this warp's rows (the same for every lane), loaded one tile ahead.
-    auto load_gates = [&](int tile, __nv_bfloat16 (&a)[kRowsT]) {
-      const int64_t tb = (int64_t)lo + (int64_t)(ch.tile0 + tile) * 128 + kRowsT * g;
-#pragma unroll
-      for (int r = 0; r < kRowsT; ++r)
-        a[r] = (tile < ch.n_tiles && tb + r < hi) ? ax[(tb + r) * H + h] : __float2bfloat16(0.f);
+    // The gate of row r of this warp's rows is computed by lanes r, r + 8, ... (its logit loaded
+    // one tile ahead; -inf past the sequence end, giving w = 0) and read by shuffles.
+    const int gl = lane & 7;
+    auto load_gate = [&](int tile) -> float {
+      const int tok = lo + (ch.tile0 + tile) * 128 + kRowsT * g + gl;
+      return (tile < ch.n_tiles && tok < hi) ? __bfloat162float(ax[(int64_t)tok * H + h]) : -INFINITY;
     };
-    __nv_bfloat16 a_next[kRowsT];
-    load_gates(0, a_next);
+    float a_next = load_gate(0);
     for (int i = 0; i < ch.n_tiles; ++i) {
-      const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
       const int s = i & 1;
       const uint32_t raw = smem_u32(ring + s * kStateStage);
-      float gate[kRowsT];
+      // Raw rows before `first` precede the sequence start (only in its first tile).
+      const int first = 3 - kRowsT * g - 128 * (ch.tile0 + i);
+      const float a = a_next;
+      a_next = load_gate(i + 1);
+      // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)).
+      const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
+      float gw_[kRowsT], glw[kRowsT];
 #pragma unroll
-      for (int r = 0; r < kRowsT; ++r)
-        gate[r] = t0 + kRowsT * g + r < hi ? sigmoidf_(__bfloat162float(a_next[r])) : 0.f;
-      load_gates(i + 1, a_next);
+      for (int r = 0; r < kRowsT; ++r) {
+        gw_[r] = __shfl_sync(0xffffffffu, w_l, r);
+        glw[r] = __shfl_sync(0xffffffffu, lw_l, r);
+      }
       ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
       // Both operand tiles are computed into registers first, then stored once the previous
       // tile's MMAs have read the operand buffers.
       uint2 uk[kRowsT], uv[kRowsT];
-      conv8(raw, sm.w[0], c4, g, t0, lo, [&](int r, float (&x)[4]) {
-        float y[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) y[e] = gate[r] * phi(x[e]);
-        uk[r] = pack4(y);
+      conv8(raw, sm.w[0], c4, g, first, [&](int r, float (&x)[4]) {
+        gated_phi2(x[0], x[1], gw_[r], glw[r]);
+        gated_phi2(x[2], x[3], gw_[r], glw[r]);
+        uk[r] = pack4(x);
       });
-      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, t0, lo, [&](int r, float (&x)[4]) { uv[r] = pack4(x); });
+      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) { uv[r] = pack4(x); });
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[0][s]);   // this warp is done with the raw tile
       if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
@@ -508,13 +535,11 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
       tmem_ld32(acc + 32 * cb, v);
       const float inv_den = 1.f / (tmem_ld1(acc + 128) + kEpsAttn);
       tc_fence_before();
-      float ssp = 0.f;
+      float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float o = __uint_as_float(v[e]) * inv_den;
-        ssp = fmaf(o, o, ssp);
-      }
-      sm.ss[cb][r] = ssp;
+      for (int e = 0; e < 32; e += 2)
+        ffma2v(s0, s1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+      sm.ss[cb][r] = (s0 + s1) * inv_den * inv_den;
       quarter_sync(qd);
       const float ss = sm.ss[0][r] + sm.ss[1][r] + sm.ss[2][r] + sm.ss[3][r];
       const float scale = inv_den * rsqrtf(ss * (1.f / 128.f) + kEpsNorm);
@@ -530,9 +555,17 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         const float4 g1 = *reinterpret_cast<const float4*>(sm.gw + 8 * chunk + 4);
         const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float zz = zf[e];
-          yv[e] = __uint_as_float(v[8 * k4 + e]) * scale * gg[e] * (zz * sigmoidf_(zz));   // silu(z)
+        for (int e = 0; e < 8; e += 2) {
+          // y = o * scale * g * silu(z), silu(z) = z (1 + tanh(z / 2)) / 2, on packed pairs.
+          float h0, h1, o0, o1;
+          fmul2v(h0, h1, zf[e], zf[e + 1], 0.5f, 0.5f);
+          h0 = tanh_approx(h0);
+          h1 = tanh_approx(h1);
+          ffma2c(h0, h1, h0, h1, 0.5f, 0.5f, 0.5f, 0.5f);
+          fmul2v(h0, h1, h0, h1, zf[e], zf[e + 1]);
+          fmul2v(h0, h1, h0, h1, gg[e], gg[e + 1]);
+          fmul2v(o0, o1, __uint_as_float(v[8 * k4 + e]), __uint_as_float(v[8 * k4 + e + 1]), scale, scale);
+          fmul2v(yv[e], yv[e + 1], h0, h1, o0, o1);
         }
         const uint4 yu = pack8(yv);
         if (whole) st_shared_v4(za, yu.x, yu.y, yu.z, yu.w);
@@ -554,16 +587,15 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
     };
 
     for (int i = 0; i < ch.n_tiles; ++i) {
-      const int64_t t0 = (int64_t)lo + (int64_t)(ch.tile0 + i) * 128;
       const int s = i & 1;
       ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
       uint2 uq[kRowsT];
-      conv8(smem_u32(qring + s * kQStage), sm.w[0], c4, g, t0, lo, [&](int rr, float (&x)[4]) {
-        float y[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) y[e] = phi(x[e]);
-        uq[rr] = pack4(y);
-      });
+      conv8(smem_u32(qring + s * kQStage), sm.w[0], c4, g, 3 - kRowsT * g - 128 * (ch.tile0 + i),
+            [&](int rr, float (&x)[4]) {
+              phi2(x[0], x[1]);
+              phi2(x[2], x[3]);
+              uq[rr] = pack4(x);
+            });
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[0][s]);
       // The previous tile's MMAs must have read A (and finished its accumulator) first.
