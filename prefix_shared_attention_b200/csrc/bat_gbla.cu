@@ -189,9 +189,8 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-// Barrier of the consumer warps (the producer warp does not take part).
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
-// Same barrier, returning whether `ok` holds in every consumer thread.
+// Barrier of the consumer warps (the producer warp does not take part), returning whether `ok`
+// holds in every consumer thread.
 __device__ __forceinline__ bool consumer_all(bool ok) {
   uint32_t r;
   asm volatile(
@@ -396,38 +395,35 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
       const int first = 3 - kRowsT * g - 128 * (ch.tile0 + i);
       const float a = a_next;
       a_next = load_gate(i + 1);
-      // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)).
+      // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)); row r's pair is read from lane r.
       const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
-      float gw_[kRowsT], glw[kRowsT];
-#pragma unroll
-      for (int r = 0; r < kRowsT; ++r) {
-        gw_[r] = __shfl_sync(0xffffffffu, w_l, r);
-        glw[r] = __shfl_sync(0xffffffffu, lw_l, r);
-      }
       ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
-      // Both operand tiles are computed into registers first, then stored once the previous
-      // tile's MMAs have read the operand buffers.
-      uint2 uk[kRowsT], uv[kRowsT];
+      // The w phi(k~) tile is computed into registers; by the time it is done the previous
+      // tile's MMAs have read the operand buffers (waited for), so it is stored and the v~ rows
+      // are stored as they are completed.
+      uint2 uk[kRowsT];
       conv8(raw, sm.w[0], c4, g, first, [&](int r, float (&x)[4]) {
-        gated_phi2(x[0], x[1], gw_[r], glw[r]);
-        gated_phi2(x[2], x[3], gw_[r], glw[r]);
+        const float wr = __shfl_sync(0xffffffffu, w_l, r), lwr = __shfl_sync(0xffffffffu, lw_l, r);
+        gated_phi2(x[0], x[1], wr, lwr);
+        gated_phi2(x[2], x[3], wr, lwr);
         uk[r] = pack4(x);
       });
-      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) { uv[r] = pack4(x); });
+      if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
+      if (ok) {
+#pragma unroll
+        for (int r = 0; r < kRowsT; ++r) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
+      }
+      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) {
+        if (ok) st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), pack4(x));
+      });
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[0][s]);   // this warp is done with the raw tile
-      if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // One barrier per tile: the operands are complete, and every thread's waits succeeded.
       if (!consumer_all(ok)) {
         ok = false;
         break;
       }
-#pragma unroll
-      for (int r = 0; r < kRowsT; ++r) {
-        st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
-        st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), uv[r]);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      consumer_sync();
       if (warp == 0) {
         tc_fence_after();
         const uint64_t ad = sdesc_sw128(smem_u32(A), kPanel, 1024), bd = sdesc_sw128(smem_u32(B), kPanel, 1024);
@@ -625,14 +621,16 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
       if (lane == 0) mbar_arrive(&sm.empty[0][s]);
       // The previous tile's MMAs must have read A (and finished its accumulator) first.
       if (ok && i > 0) ok = wait_phase(&sm.mma_done[(i - 1) & 1], ((i - 1) >> 1) & 1, sm, p.status);
+      if (ok) {
+#pragma unroll
+        for (int rr = 0; rr < kRowsT; ++rr) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + rr, c4), uq[rr]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // One barrier per tile: A is complete, and every thread's waits succeeded.
       if (!consumer_all(ok)) {
         ok = false;
         break;
       }
-#pragma unroll
-      for (int rr = 0; rr < kRowsT; ++rr) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + rr, c4), uq[rr]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      consumer_sync();
       if (warp == 0) {
         tc_fence_after();
         const uint64_t ad = sdesc_sw128(smem_u32(A), 16, 1024), bd = sdesc_sw128(smem_u32(Bs), kPanel, 1024);
