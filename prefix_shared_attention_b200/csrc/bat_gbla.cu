@@ -92,7 +92,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 
 struct GblaSmem {
   float w[2][4 * 128];              // convolution taps (state: k, v; output: q)
-  float gw[128];                    // output: norm weight
+  float gw[128];                    // output: half the norm weight
   float ss[4][128];                 // output: partial sums of squares of each row, per 32-column block
   uint64_t full[2][2], empty[2][2];   // [ring][stage]
   uint64_t mma_done[2];             // per accumulator (the state kernel uses one)
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
   // n as the first column of the third panel: the MMA's column d is n . phi(q~).
   if (tid < 128) write_extra_row(Bs + 2 * kPanel, tid, p.norm_n[(int64_t)ch.pair * 128 + tid]);
   for (int i = tid; i < 4 * 128; i += kThreads) sm.w[0][i] = p.conv_q[h * 4 * 128 + i];
-  if (tid < 128) sm.gw[tid] = p.norm_w[h * 128 + tid];
+  if (tid < 128) sm.gw[tid] = 0.5f * p.norm_w[h * 128 + tid];   // g / 2 (see the epilogue)
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
@@ -577,14 +577,14 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-          // y = o * scale * g * silu(z), silu(z) = z (1 + tanh(z / 2)) / 2, on packed pairs.
-          float h0, h1, o0, o1;
+          // y = o * scale * g * silu(z) with g * silu(z) = u + u tanh(z / 2), u = z g / 2 (the
+          // shared memory holds g / 2), on packed pairs.
+          float u0, u1, h0, h1, o0, o1;
+          fmul2v(u0, u1, zf[e], zf[e + 1], gg[e], gg[e + 1]);
           fmul2v(h0, h1, zf[e], zf[e + 1], 0.5f, 0.5f);
           h0 = tanh_approx(h0);
           h1 = tanh_approx(h1);
-          ffma2c(h0, h1, h0, h1, 0.5f, 0.5f, 0.5f, 0.5f);
-          fmul2v(h0, h1, h0, h1, zf[e], zf[e + 1]);
-          fmul2v(h0, h1, h0, h1, gg[e], gg[e + 1]);
+          ffma2c(h0, h1, h0, h1, u0, u1, u0, u1);
           fmul2v(o0, o1, __uint_as_float(v[8 * k4 + e]), __uint_as_float(v[8 * k4 + e + 1]), scale, scale);
           fmul2v(yv[e], yv[e + 1], h0, h1, o0, o1);
         }
