@@ -108,6 +108,8 @@ int32_t debug_shrink() {
 namespace bat {
 // Sets this thread's bat_last_error() message (for entry points defined in other files).
 void set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+// The spin-wait limit set by bat_set_wait_timeout_ns (for kernels launched from other files).
+uint64_t wait_limit_ns() { return g_wait_ns.load(); }
 }  // namespace bat
 
 extern "C" {

@@ -14,9 +14,10 @@
 // producer warp loads 128-token tiles (plus the 8 rows before them, for the convolution) into
 // two-stage rings with TMA; sixteen consumer warps read them from shared memory (each thread 8
 // consecutive rows x 4 channels, so the convolution reads 11 raw rows per 8 outputs), apply the
-// convolution, feature map and gate in fp32 registers, write bf16 operand tiles in the 128-byte-
-// swizzled layout, and one elected thread issues the tile's tcgen05.mma.  The next tiles' loads
-// are in flight while a tile is computed.
+// convolution, feature map and gate in fp32 registers, write 16-bit operand tiles (fp16 for
+// the state contraction, bf16 for the output one) in the 128-byte-swizzled layout, and one
+// elected thread issues the tile's tcgen05.mma.  The next tiles' loads are in flight while a
+// tile is computed.
 //   gbla_state_kernel   per chunk (consecutive tiles of one (sequence, head)):
 //                       D[d x (d+16)] += (w phi(k~))^T [v~ | 1] (M = d, N = d + 16, K = tokens;
 //                       both operands MN-major; the ones column gives n); the partial state and
@@ -32,6 +33,7 @@
 // once and y is written once; S and the partials stay small and in L2.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -88,7 +90,9 @@ constexpr uint32_t kAccStride = 256;          // TMEM columns between the output
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kEpsAttn = 1e-6f;
 constexpr float kEpsNorm = 1e-6f;
-constexpr uint64_t kWaitNs = 2000000000ull;
+// Upper bound on the waits that let in-flight copies and MMAs finish before a CTA that is
+// aborting releases its shared memory and tensor memory (independent of the wait limit).
+constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 struct GblaSmem {
   float w[2][4 * 128];              // convolution taps (state: k, v; output: q)
@@ -96,6 +100,7 @@ struct GblaSmem {
   float ss[4][128];                 // output: partial sums of squares of each row, per 32-column block
   uint64_t full[2][2], empty[2][2];   // [ring][stage]
   uint64_t mma_done[2];             // per accumulator (the state kernel uses one)
+  uint64_t wait_ns;                 // bound on every wait (the launch's wait limit)
   uint32_t tmem_slot;
   int abort;
 };
@@ -156,6 +161,13 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
 __device__ __forceinline__ uint2 pack4(const float (&v)[4]) {
   return make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);   // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint2 pack4h(const float (&v)[4]) {
+  return make_uint2(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]));
+}
 __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
   uint4 u;
   u.x = pack_bf16x2(v[0], v[1]);
@@ -203,13 +215,17 @@ __device__ __forceinline__ bool consumer_all(bool ok) {
 // Barrier of the four consumer warps that read TMEM lane quarter qd (warps qd, qd+4, qd+8, qd+12).
 __device__ __forceinline__ void quarter_sync(int qd) { asm volatile("bar.sync %0, 128;" ::"r"(2 + qd) : "memory"); }
 
-// Bounded wait on an mbarrier phase; false on timeout or when the CTA is aborting.
+// Bounded wait on an mbarrier phase; false on timeout or when the CTA is aborting.  The first
+// probe does not block; later probes suspend for at most 1 ms, and not at all under a limit
+// below 100 us (a suspended probe may outlast a hint that short), so the limit is always seen.
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, GblaSmem& sm, uint32_t* status) {
   if (mbar_test(bar, parity)) return true;
+  const uint64_t limit = sm.wait_ns;
+  const bool spin = limit < 100000ull;
   const uint64_t t0 = global_ns();
-  while (!mbar_test_suspend(bar, parity, 1000000u)) {
+  while (!(spin ? mbar_test(bar, parity) : mbar_test_suspend(bar, parity, 1000000u))) {
     if (*reinterpret_cast<volatile int*>(&sm.abort)) return false;
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > limit) {
       atomicOr(status, 1u);
       *reinterpret_cast<volatile int*>(&sm.abort) = 1;
       return false;
@@ -222,7 +238,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, GblaS
 __device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
   while (!mbar_test(bar, parity))
-    if (global_ns() - t0 > kWaitNs / 10) break;
+    if (global_ns() - t0 > kDrainNs) break;
 }
 
 // The causal convolution (width 4) of this thread's 8 rows (8g .. 8g+7 of the tile) and 4
@@ -318,7 +334,7 @@ __device__ __forceinline__ void produce(const GblaChunk& ch, GblaSmem& sm, const
   __syncwarp();
 }
 
-__device__ __forceinline__ void init_barriers(GblaSmem& sm, int nrings) {
+__device__ __forceinline__ void init_barriers(GblaSmem& sm, int nrings, uint64_t wait_ns) {
   for (int q = 0; q < nrings; ++q)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.full[q][s], 1);
@@ -327,15 +343,16 @@ __device__ __forceinline__ void init_barriers(GblaSmem& sm, int nrings) {
   mbar_init(&sm.mma_done[0], 1);
   mbar_init(&sm.mma_done[1], 1);
   sm.abort = 0;
+  sm.wait_ns = wait_ns;
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// Row r of the third (64-column) panel of a 128-row operand tile: value x in its first column,
-// zeros elsewhere.
-__device__ __forceinline__ void write_extra_row(uint8_t* panel, int r, float x) {
+// Row r of the third (64-column) panel of a 128-row operand tile: value x in its first column
+// (fp16 or bf16), zeros elsewhere.
+__device__ __forceinline__ void write_extra_row(uint8_t* panel, int r, float x, bool f16) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint32_t v0 = k == 0 ? pack_bf16x2(x, 0.f) : 0u;
+    const uint32_t v0 = k == 0 ? (f16 ? pack_f16x2(x, 0.f) : pack_bf16x2(x, 0.f)) : 0u;
     st_shared_v4(smem_u32(panel) + r * 128 + ((k ^ (r & 7)) << 4), v0, 0u, 0u, 0u);
   }
 }
@@ -353,13 +370,13 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
   const GblaChunk ch = p.chunks[blockIdx.x];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
-  if (tid == 0) init_barriers(sm, 1);
+  if (tid == 0) init_barriers(sm, 1, p.wait_ns);
   for (int i = tid; i < 4 * 128; i += kThreads) {
     sm.w[0][i] = p.conv_k[h * 4 * 128 + i];
     sm.w[1][i] = p.conv_v[h * 4 * 128 + i];
   }
   // The ones column: n = sum over tokens of w phi(k~) comes out of the MMA as column d.
-  if (tid < 128) write_extra_row(B + 2 * kPanel, tid, 1.f);
+  if (tid < 128) write_extra_row(B + 2 * kPanel, tid, 1.f, true);
   if (warp == 0) tmem_alloc(&sm.tmem_slot, 256);
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&p.tm_k);
@@ -377,7 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
   } else {
     const int g = warp, c4 = lane;
     const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
-    constexpr uint32_t idesc = make_idesc(128, kN, true, true);
+    // fp16 operands (A and B of one type, as kind::f16 requires): the rounding of w phi(k~) and
+    // v~ is the largest error of the layer (the output's RMS normalisation magnifies it in rows
+    // whose weighted average nearly cancels), and fp16 has 3 more mantissa bits than bf16; both
+    // stay far inside its range (|w phi(k~)|, |v~| < 65504).
+    constexpr uint32_t idesc = make_idesc(128, kN, true, true) & ~((7u << 7) | (7u << 10));
     bool ok = true;
     int done = 0;
     // The gate of row r of this warp's rows is computed by lanes r, r + 8, ... (its logit loaded
@@ -397,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
       a_next = load_gate(i + 1);
       // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)); row r's pair is read from lane r.
       const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
-      ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      const bool landed = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      ok = landed;
       // The w phi(k~) tile is computed into registers; by the time it is done the previous
       // tile's MMAs have read the operand buffers (waited for), so it is stored and the v~ rows
       // are stored as they are completed.
@@ -406,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
         const float wr = __shfl_sync(0xffffffffu, w_l, r), lwr = __shfl_sync(0xffffffffu, lw_l, r);
         gated_phi2(x[0], x[1], wr, lwr);
         gated_phi2(x[2], x[3], wr, lwr);
-        uk[r] = pack4(x);
+        uk[r] = pack4h(x);
       });
       if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
       if (ok) {
@@ -414,10 +436,11 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
         for (int r = 0; r < kRowsT; ++r) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
       }
       conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) {
-        if (ok) st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), pack4(x));
+        if (ok) st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), pack4h(x));
       });
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[0][s]);   // this warp is done with the raw tile
+      // This warp is done with the raw tile (released only if it saw the tile land: a stage
+      // whose copy may still be in flight is never handed back to the producer).
+      if (__all_sync(0xffffffffu, landed) && lane == 0) mbar_arrive(&sm.empty[0][s]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       // One barrier per tile: the operands are complete, and every thread's waits succeeded.
       if (!consumer_all(ok)) {
@@ -499,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
   const GblaChunk ch = p.chunks[blockIdx.x];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
-  if (tid == 0) init_barriers(sm, 2);
+  if (tid == 0) init_barriers(sm, 2, p.wait_ns);
   if (warp == 0) tmem_alloc(&sm.tmem_slot, 512);
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&p.tm_q);
@@ -516,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
     }
   }
   // n as the first column of the third panel: the MMA's column d is n . phi(q~).
-  if (tid < 128) write_extra_row(Bs + 2 * kPanel, tid, p.norm_n[(int64_t)ch.pair * 128 + tid]);
+  if (tid < 128) write_extra_row(Bs + 2 * kPanel, tid, p.norm_n[(int64_t)ch.pair * 128 + tid], false);
   for (int i = tid; i < 4 * 128; i += kThreads) sm.w[0][i] = p.conv_q[h * 4 * 128 + i];
   if (tid < 128) sm.gw[tid] = 0.5f * p.norm_w[h * 128 + tid];   // g / 2 (see the epilogue)
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -603,13 +626,13 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         bulk_wait_read();
         stores_pending = true;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[1][zs]);
+      if (__all_sync(0xffffffffu, zok) && lane == 0) mbar_arrive(&sm.empty[1][zs]);
     };
 
     for (int i = 0; i < ch.n_tiles; ++i) {
       const int s = i & 1;
-      ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      const bool landed = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+      ok = landed;
       uint2 uq[kRowsT];
       conv8(smem_u32(qring + s * kQStage), sm.w[0], c4, g, 3 - kRowsT * g - 128 * (ch.tile0 + i),
             [&](int rr, float (&x)[4]) {
@@ -617,8 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
               phi2(x[2], x[3]);
               uq[rr] = pack4(x);
             });
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[0][s]);
+      if (__all_sync(0xffffffffu, landed) && lane == 0) mbar_arrive(&sm.empty[0][s]);
       // The previous tile's MMAs must have read A (and finished its accumulator) first.
       if (ok && i > 0) ok = wait_phase(&sm.mma_done[(i - 1) & 1], ((i - 1) >> 1) & 1, sm, p.status);
       if (ok) {

@@ -266,6 +266,7 @@ bat_status bat_gbla_forward(const bat_gbla_plan* plan, const void* q, const void
   p.norm_n = reinterpret_cast<float*>(ws + align256(nc * kPartFloats * 4) + align256(np * 128 * 128 * 2));
   p.H = plan->H;
   p.status = status;
+  p.wait_ns = bat::wait_limit_ns();
   e = bat::launch_gbla(p, (int)nc, (int)np, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     char buf[200];

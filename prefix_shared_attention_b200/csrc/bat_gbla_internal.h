@@ -47,8 +47,10 @@ struct alignas(64) GblaParams {
   int32_t H;
   int32_t pad;
   uint32_t* status;         // device status word (bit 0: a wait timed out)
+  uint64_t wait_ns;         // bound on every spin-wait (bat_set_wait_timeout_ns)
 };
 
 cudaError_t launch_gbla(const GblaParams& p, int n_chunks, int n_pairs, cudaStream_t s);
+uint64_t wait_limit_ns();   // the current bat_set_wait_timeout_ns setting
 
 }  // namespace bat

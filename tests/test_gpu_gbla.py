@@ -91,3 +91,26 @@ def test_gbla_long_history_sampled():
     rows = np.sort(np.random.default_rng(5).choice(so[-1], 256, replace=False))
     ref = oracle_y(x, so, rows)
     check(y.float().cpu().numpy()[rows], ref, "long history")
+
+
+def test_gbla_wait_timeout_reports_and_context_survives():
+    """Failure detection on the GBLA kernels: with a 1 ns wait limit the first wait whose phase
+    has not completed (a tile that has not landed yet) runs out, the kernels abort (their copies
+    and MMAs in flight drained, tensor memory freed), the status word reports BAT_ERR_TIMEOUT,
+    and the next run on the same context is correct."""
+    lens, H = [3000, 2000], 2
+    x, so = make_inputs(lens, H, seed=21)
+    xd = {k: v.cuda().contiguous() for k, v in x.items()}
+    bat.bat_set_wait_timeout_ns(1)
+    try:
+        with bat.GblaPlan(so, H) as plan:
+            y = torch.empty_like(xd["q"])
+            bat.bat_gbla_forward(plan, xd["q"], xd["k"], xd["v"], xd["a"], xd["z"], xd["cq"], xd["ck"], xd["cv"], xd["g"],
+                                 y=y)
+            st = bat.bat_get_device_status()
+    finally:
+        bat.bat_set_wait_timeout_ns(0)
+    assert st == bat.BAT_ERR_TIMEOUT, f"expected BAT_ERR_TIMEOUT, got {st}: {bat.last_error()}"
+    y = run_gpu(x, so, H)
+    check(y.float().cpu().numpy(), oracle_y(x, so), "after a timed-out run")
+    assert bat.bat_get_device_status() == bat.BAT_OK
