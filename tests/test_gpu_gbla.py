@@ -5,9 +5,11 @@ Bar, derived from the arithmetic.  y is stored in bf16 and its entries are not s
 has unit RMS before the gates, times g * silu(z), so |y| reaches ~15, where one bf16 rounding
 alone is up to 2^-5.  The elementwise bound is therefore relative plus absolute:
 |gpu - ref| <= 2e-2 + 1e-2 |ref|, from at most about 1 % accumulated relative error: the bf16
-roundings of y (2^-9), of S and of phi(q~) (2^-9 each, entering o directly) and of the state
-operands (averaged over the tokens), with margin.  The aggregate bar is the attention path's:
-sum|gpu - ref| / sum|ref| <= 5e-3.
+roundings of y (2^-9), of S and of phi(q~) (2^-9 each, entering o directly) and the fp16
+roundings of the state operands w phi(k~) and v~ (2^-11 each; they do not simply average out
+over the tokens: the RMS normalisation divides by the row's own output, so a row whose
+weighted average nearly cancels magnifies them, which is why they are fp16 and not bf16), with
+margin.  The aggregate bar is the attention path's: sum|gpu - ref| / sum|ref| <= 5e-3.
 
 Ragged sequence lengths cover empty sequences, one token, tile multiples +-1 and several tiles
 per chunk; guard rows around y must stay untouched; a long history (the bench workload's
