@@ -10,9 +10,10 @@
 //   o[t] = S^T phi(q~[t]) / (n . phi(q~[t]) + 1e-6),   phi(x) = elu(x) + 1
 //   y[t] = o[t] / sqrt(mean(o[t]^2) + 1e-6) * g * silu(z[t])
 //
-// Three kernels; the two that stream the tokens are pipelined alike.  One CTA per SM: a
-// producer warp loads 128-token tiles (plus the 8 rows before them, for the convolution) into
-// two-stage rings with TMA; sixteen consumer warps read them from shared memory (each thread 8
+// Three kernels; the two that stream the tokens are pipelined alike.  One CTA per SM: 128-token
+// tiles (plus the 8 rows before them, for the convolution) arrive by TMA in two-stage rings
+// (issued by thread 0 in the state kernel, by a producer warp in the output kernel, whose two
+// rings drain at different times); sixteen warps read them from shared memory (each thread 8
 // consecutive rows x 4 channels, so the convolution reads 11 raw rows per 8 outputs), apply the
 // convolution, feature map and gate in fp32 registers, write 16-bit operand tiles (fp16 for
 // the state contraction, bf16 for the output one) in the 128-byte-swizzled layout, and one
@@ -358,9 +359,11 @@ __device__ __forceinline__ void write_extra_row(uint8_t* panel, int r, float x, 
 }
 
 // ---------------------------------------------------------------------------------------
-// State: partial S and n of one chunk.
+// State: partial S and n of one chunk.  No producer warp: 16 warps (so up to 128 registers per
+// thread); thread 0 issues the loads of tile i + 2 into the stage tile i used once the tile's
+// barrier has shown every warp done with it.
 
-__global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_constant__ GblaParams p) {
+__global__ void __launch_bounds__(kConsumers, 1) gbla_state_kernel(const __grid_constant__ GblaParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* A = base;                // (w phi(k~)) tile: rows = tokens, columns = d (MN-major A)
@@ -371,118 +374,130 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_state_kernel(const __grid_co
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
   if (tid == 0) init_barriers(sm, 1, p.wait_ns);
-  for (int i = tid; i < 4 * 128; i += kThreads) {
+  for (int i = tid; i < 4 * 128; i += kConsumers) {
     sm.w[0][i] = p.conv_k[h * 4 * 128 + i];
     sm.w[1][i] = p.conv_v[h * 4 * 128 + i];
   }
   // The ones column: n = sum over tokens of w phi(k~) comes out of the MMA as column d.
   if (tid < 128) write_extra_row(B + 2 * kPanel, tid, 1.f, true);
   if (warp == 0) tmem_alloc(&sm.tmem_slot, 256);
-  if (warp == kProducerWarp && lane == 0) {
-    prefetch_tmap(&p.tm_k);
-    prefetch_tmap(&p.tm_v);
-  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
-
-  if (warp == kProducerWarp) {
-    const Ring r0 = {{&p.tm_k, &p.tm_v}, 2, 8, kRawPanel, kStateStage, ring, sm.full[0], sm.empty[0]};
-    produce(ch, sm, &r0, 1, p.status);
-  } else {
-    const int g = warp, c4 = lane;
-    const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
-    // fp16 operands (A and B of one type, as kind::f16 requires): the rounding of w phi(k~) and
-    // v~ is the largest error of the layer (the output's RMS normalisation magnifies it in rows
-    // whose weighted average nearly cancels), and fp16 has 3 more mantissa bits than bf16; both
-    // stay far inside its range (|w phi(k~)|, |v~| < 65504).
-    constexpr uint32_t idesc = make_idesc(128, kN, true, true) & ~((7u << 7) | (7u << 10));
-    bool ok = true;
-    int done = 0;
-    // The gate of row r of this warp's rows is computed by lanes r, r + 8, ... (its logit loaded
-    // one tile ahead; -inf past the sequence end, giving w = 0) and read by shuffles.
-    const int gl = lane & 7;
-    auto load_gate = [&](int tile) -> float {
-      const int tok = lo + (ch.tile0 + tile) * 128 + kRowsT * g + gl;
-      return (tile < ch.n_tiles && tok < hi) ? __bfloat162float(ax[(int64_t)tok * H + h]) : -INFINITY;
-    };
-    float a_next = load_gate(0);
-    for (int i = 0; i < ch.n_tiles; ++i) {
-      const int s = i & 1;
-      const uint32_t raw = smem_u32(ring + s * kStateStage);
-      // Raw rows before `first` precede the sequence start (only in its first tile).
-      const int first = 3 - kRowsT * g - 128 * (ch.tile0 + i);
-      const float a = a_next;
-      a_next = load_gate(i + 1);
-      // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)); row r's pair is read from lane r.
-      const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
-      const bool landed = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
-      ok = landed;
-      // The w phi(k~) tile is computed into registers; by the time it is done the previous
-      // tile's MMAs have read the operand buffers (waited for), so it is stored and the v~ rows
-      // are stored as they are completed.
-      uint2 uk[kRowsT];
-      conv8(raw, sm.w[0], c4, g, first, [&](int r, float (&x)[4]) {
-        const float wr = __shfl_sync(0xffffffffu, w_l, r), lwr = __shfl_sync(0xffffffffu, lw_l, r);
-        gated_phi2(x[0], x[1], wr, lwr);
-        gated_phi2(x[2], x[3], wr, lwr);
-        uk[r] = pack4h(x);
-      });
-      if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
-      if (ok) {
+  // Tile t's k and v (two panels each, from 8 rows before the tile) into stage t % 2.
+  auto issue = [&](int t) {
+    const int s = t & 1, y0 = ch.seq_lo + (ch.tile0 + t) * 128;
+    uint8_t* st = ring + s * kStateStage;
+    mbar_expect_tx(&sm.full[0][s], kStateStage);
 #pragma unroll
-        for (int r = 0; r < kRowsT; ++r) st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
-      }
-      conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) {
-        if (ok) st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), pack4h(x));
-      });
-      // This warp is done with the raw tile (released only if it saw the tile land: a stage
-      // whose copy may still be in flight is never handed back to the producer).
-      if (__all_sync(0xffffffffu, landed) && lane == 0) mbar_arrive(&sm.empty[0][s]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      // One barrier per tile: the operands are complete, and every thread's waits succeeded.
-      if (!consumer_all(ok)) {
-        ok = false;
-        break;
-      }
-      if (warp == 0) {
-        tc_fence_after();
-        const uint64_t ad = sdesc_sw128(smem_u32(A), kPanel, 1024), bd = sdesc_sw128(smem_u32(B), kPanel, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // 16 tokens per step: two 8-row swizzle groups (2 KiB)
-          mma_ss_w(tmem, ad + (uint64_t)(kk * 2048 / 16), bd + (uint64_t)(kk * 2048 / 16), idesc,
-                   (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit_w(&sm.mma_done[0]);
-      }
-      done = i + 1;
+    for (int pn = 0; pn < 2; ++pn) {
+      tma_load_2d(st + pn * kRawPanel, &p.tm_k, h * 128 + pn * 64, y0 - 8, &sm.full[0][s]);
+      tma_load_2d(st + (2 + pn) * kRawPanel, &p.tm_v, h * 128 + pn * 64, y0 - 8, &sm.full[0][s]);
     }
-    if (done > 0) {
-      if (ok) ok = wait_phase(&sm.mma_done[0], (done - 1) & 1, sm, p.status);
-      else drain_phase(&sm.mma_done[0], (done - 1) & 1);
-    }
-    ok = consumer_all(ok);
-    tc_fence_after();
-    float* part = p.part_s + (int64_t)blockIdx.x * (128 * 128 + 128);
-    {
-      // Row i = 32 * (warp % 4) + lane of the partial state (channel i of phi(k~)), columns
-      // 32 * (warp / 4) .. +31 (v channels): one 32-column TMEM load per warp; column d is n.
-      const int qd = warp & 3, cb = warp >> 2;
-      const int i = 32 * qd + lane;
-      const bool keep = ok && done > 0;
-      float4* dst = reinterpret_cast<float4*>(part + (int64_t)i * 128 + 32 * cb);
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * cb, r);
+  };
+  int issued = 0;
+  if (tid == 0) {
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+    for (; issued < 2 && issued < ch.n_tiles; ++issued) issue(issued);
+  }
+  const int g = warp, c4 = lane;
+  const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
+  // fp16 operands (A and B of one type, as kind::f16 requires): the rounding of w phi(k~) and
+  // v~ is the largest error of the layer (the output's RMS normalisation magnifies it in rows
+  // whose weighted average nearly cancels), and fp16 has 3 more mantissa bits than bf16; both
+  // stay far inside its range (|w phi(k~)|, |v~| < 65504).
+  constexpr uint32_t idesc = make_idesc(128, kN, true, true) & ~((7u << 7) | (7u << 10));
+  bool ok = true;
+  int done = 0;
+  // The gate of row r of this warp's rows is computed by lanes r, r + 8, ... (its logit loaded
+  // one tile ahead; -inf past the sequence end, giving w = 0) and read by shuffles.
+  const int gl = lane & 7;
+  auto load_gate = [&](int tile) -> float {
+    const int tok = lo + (ch.tile0 + tile) * 128 + kRowsT * g + gl;
+    return (tile < ch.n_tiles && tok < hi) ? __bfloat162float(ax[(int64_t)tok * H + h]) : -INFINITY;
+  };
+  float a_next = load_gate(0);
+  for (int i = 0; i < ch.n_tiles; ++i) {
+    const int s = i & 1;
+    const uint32_t raw = smem_u32(ring + s * kStateStage);
+    // Raw rows before `first` precede the sequence start (only in its first tile).
+    const int first = 3 - kRowsT * g - 128 * (ch.tile0 + i);
+    const float a = a_next;
+    a_next = load_gate(i + 1);
+    // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)); row r's pair is read from lane r.
+    const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
+    ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
+    uint2 uk[kRowsT], uv[kRowsT];
+    // Both operand tiles into registers first (no wait between the two convolutions, so they
+    // can interleave), then stored once the previous tile's MMAs have read the buffers.
+    conv8(raw, sm.w[0], c4, g, first, [&](int r, float (&x)[4]) {
+      const float wr = __shfl_sync(0xffffffffu, w_l, r), lwr = __shfl_sync(0xffffffffu, lw_l, r);
+      gated_phi2(x[0], x[1], wr, lwr);
+      gated_phi2(x[2], x[3], wr, lwr);
+      uk[r] = pack4h(x);
+    });
+    conv8(raw + 2 * kRawPanel, sm.w[1], c4, g, first, [&](int r, float (&x)[4]) { uv[r] = pack4h(x); });
+    if (ok && i > 0) ok = wait_phase(&sm.mma_done[0], (i - 1) & 1, sm, p.status);
+    if (ok) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        dst[e] = keep ? make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                                    __uint_as_float(r[4 * e + 3]))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      if (cb == 0) {
-        const float nv = tmem_ld1(tmem + ((uint32_t)(32 * qd) << 16) + 128);
-        part[128 * 128 + i] = keep ? nv : 0.f;
+      for (int r = 0; r < kRowsT; ++r) {
+        st_shared_v2(smem_u32(A) + sw_off8(kRowsT * g + r, c4), uk[r]);
+        st_shared_v2(smem_u32(B) + sw_off8(kRowsT * g + r, c4), uv[r]);
       }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    // One barrier per tile: the operands are complete, every thread's waits succeeded, and no
+    // warp reads stage s any more.
+    if (!consumer_all(ok)) {
+      ok = false;
+      break;
+    }
+    if (warp == 0) {
+      if (lane == 0 && i + 2 < ch.n_tiles) {
+        issue(i + 2);
+        ++issued;
+      }
+      tc_fence_after();
+      const uint64_t ad = sdesc_sw128(smem_u32(A), kPanel, 1024), bd = sdesc_sw128(smem_u32(B), kPanel, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss_w(tmem, ad + (uint64_t)(kk * 2048 / 16), bd + (uint64_t)(kk * 2048 / 16), idesc,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+      tc_commit_w(&sm.mma_done[0]);
+    }
+    done = i + 1;
+  }
+  if (tid == 0 && !ok) {
+    // Aborting: let the loads in flight land before the CTA releases its shared memory.
+    for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t) drain_phase(&sm.full[0][t & 1], (t >> 1) & 1);
+  }
+  if (done > 0) {
+    if (ok) ok = wait_phase(&sm.mma_done[0], (done - 1) & 1, sm, p.status);
+    else drain_phase(&sm.mma_done[0], (done - 1) & 1);
+  }
+  ok = consumer_all(ok);
+  tc_fence_after();
+  float* part = p.part_s + (int64_t)blockIdx.x * (128 * 128 + 128);
+  {
+    // Row i = 32 * (warp % 4) + lane of the partial state (channel i of phi(k~)), columns
+    // 32 * (warp / 4) .. +31 (v channels): one 32-column TMEM load per warp; column d is n.
+    const int qd = warp & 3, cb = warp >> 2;
+    const int i = 32 * qd + lane;
+    const bool keep = ok && done > 0;
+    float4* dst = reinterpret_cast<float4*>(part + (int64_t)i * 128 + 32 * cb);
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * cb, r);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      dst[e] = keep ? make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                                  __uint_as_float(r[4 * e + 3]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (cb == 0) {
+      const float nv = tmem_ld1(tmem + ((uint32_t)(32 * qd) << 16) + 128);
+      part[128 * 128 + i] = keep ? nv : 0.f;
     }
   }
   tc_fence_before();
@@ -687,7 +702,7 @@ cudaError_t launch_gbla(const GblaParams& p, int n_chunks, int n_pairs, cudaStre
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(gbla_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
   if (e != cudaSuccess) return e;
-  gbla_state_kernel<<<n_chunks, kThreads, kStateSmem, s>>>(p);
+  gbla_state_kernel<<<n_chunks, kConsumers, kStateSmem, s>>>(p);
   gbla_reduce_kernel<<<dim3(n_pairs, (128 * 128 + 128 + 255) / 256), 256, 0, s>>>(p);
   gbla_out_kernel<<<n_chunks, kThreads, kOutSmem, s>>>(p);
   return cudaGetLastError();
