@@ -10,10 +10,10 @@
 //   o[t] = S^T phi(q~[t]) / (n . phi(q~[t]) + 1e-6),   phi(x) = elu(x) + 1
 //   y[t] = o[t] / sqrt(mean(o[t]^2) + 1e-6) * g * silu(z[t])
 //
-// Three kernels; the two that stream the tokens are pipelined alike.  One CTA per SM: 128-token
-// tiles (plus the 8 rows before them, for the convolution) arrive by TMA in two-stage rings
-// (issued by thread 0 in the state kernel, by a producer warp in the output kernel, whose two
-// rings drain at different times); sixteen warps read them from shared memory (each thread 8
+// Three kernels; the two that stream the tokens are pipelined alike.  One CTA of 16 warps per
+// SM: 128-token tiles (plus the 8 rows before them, for the convolution) arrive by TMA in
+// two-stage rings, issued by thread 0 right after the tile barrier that shows every warp done
+// with the stage; the warps read them from shared memory (each thread 8
 // consecutive rows x 4 channels, so the convolution reads 11 raw rows per 8 outputs), apply the
 // convolution, feature map and gate in fp32 registers, write 16-bit operand tiles (fp16 for
 // the state contraction, bf16 for the output one) in the 128-byte-swizzled layout, and one
@@ -72,9 +72,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
 }
 
 constexpr int kConsumerWarps = 16;
-constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kThreads = kConsumers + 32;     // plus the producer warp (warp 16)
-constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kConsumers = 32 * kConsumerWarps;   // every thread of a CTA
 // Consumer thread (warp w, lane l): rows 8w .. 8w+7 of a tile, channels 4l .. 4l+3.
 constexpr int kRowsT = 8;
 constexpr int kPanel = 128 * 128;             // one 64-column panel of a 128-row bf16 tile
@@ -99,7 +97,7 @@ struct GblaSmem {
   float w[2][4 * 128];              // convolution taps (state: k, v; output: q)
   float gw[128];                    // output: half the norm weight
   float ss[4][128];                 // output: partial sums of squares of each row, per 32-column block
-  uint64_t full[2][2], empty[2][2];   // [ring][stage]
+  uint64_t full[2][2];              // [ring][stage]: the stage's copies have landed
   uint64_t mma_done[2];             // per accumulator (the state kernel uses one)
   uint64_t wait_ns;                 // bound on every wait (the launch's wait limit)
   uint32_t tmem_slot;
@@ -202,8 +200,7 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-// Barrier of the consumer warps (the producer warp does not take part), returning whether `ok`
-// holds in every consumer thread.
+// Barrier of all 16 warps, returning whether `ok` holds in every thread.
 __device__ __forceinline__ bool consumer_all(bool ok) {
   uint32_t r;
   asm volatile(
@@ -289,58 +286,9 @@ __device__ __forceinline__ void tmem_free(uint32_t tmem, uint32_t cols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols) : "memory");
 }
 
-// A two-stage ring of tiles filled by the producer warp: `nmaps` tensors per stage, each as two
-// 64-column panels of `panel` bytes starting `before` rows before the tile.
-struct Ring {
-  const CUtensorMap* map[2];
-  int nmaps, before, panel, stage;
-  uint8_t* base;
-  uint64_t *full, *empty;
-};
-
-// Producer warp: tile i of the chunk into stage i % 2 of every ring, in ring order; drains its
-// loads if the CTA aborts.
-__device__ __forceinline__ void produce(const GblaChunk& ch, GblaSmem& sm, const Ring* rings, int nrings,
-                                        uint32_t* status) {
-  const int lane = threadIdx.x & 31;
-  int issued[2] = {0, 0};
-  bool ok = true;
-  for (int i = 0; ok && i < ch.n_tiles; ++i) {
-    const int s = i & 1;
-    for (int q = 0; q < nrings; ++q) {
-      const Ring& R = rings[q];
-      if (!wait_phase(&R.empty[s], ((i >> 1) & 1) ^ 1, sm, status)) {
-        ok = false;
-        break;
-      }
-      if (lane == 0) {
-        const int y0 = ch.seq_lo + (ch.tile0 + i) * 128;
-        mbar_expect_tx(&R.full[s], R.stage);
-        for (int m = 0; m < R.nmaps; ++m)
-#pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_2d(R.base + s * R.stage + (2 * m + pn) * R.panel, R.map[m], ch.head * 128 + pn * 64, y0 - R.before,
-                        &R.full[s]);
-      }
-      __syncwarp();
-      ++issued[q];
-    }
-  }
-  if (!ok && lane == 0) {
-    // Aborting: let the loads in flight land before the CTA releases its shared memory.
-    for (int q = 0; q < nrings; ++q)
-      for (int i = (issued[q] > 2 ? issued[q] - 2 : 0); i < issued[q]; ++i)
-        drain_phase(&rings[q].full[i & 1], (i >> 1) & 1);
-  }
-  __syncwarp();
-}
-
 __device__ __forceinline__ void init_barriers(GblaSmem& sm, int nrings, uint64_t wait_ns) {
   for (int q = 0; q < nrings; ++q)
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.full[q][s], 1);
-      mbar_init(&sm.empty[q][s], kConsumerWarps);   // one arrival per consumer warp
-    }
+    for (int s = 0; s < 2; ++s) mbar_init(&sm.full[q][s], 1);   // thread 0's arrival + the copies' bytes
   mbar_init(&sm.mma_done[0], 1);
   mbar_init(&sm.mma_done[1], 1);
   sm.abort = 0;
@@ -526,7 +474,7 @@ __global__ void __launch_bounds__(256) gbla_reduce_kernel(const __grid_constant_
 // i - 1 reads the other TMEM accumulator; q and z come through separate rings because z is
 // needed one tile later than q.
 
-__global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_constant__ GblaParams p) {
+__global__ void __launch_bounds__(kConsumers, 1) gbla_out_kernel(const __grid_constant__ GblaParams p) {
   extern __shared__ uint8_t dyn[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* A = base;                 // phi(q~) tile: rows = tokens, columns = d (K-major A)
@@ -539,12 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
   const int h = ch.head, lo = ch.seq_lo, hi = ch.seq_hi, H = p.H;
   if (tid == 0) init_barriers(sm, 2, p.wait_ns);
   if (warp == 0) tmem_alloc(&sm.tmem_slot, 512);
-  if (warp == kProducerWarp && lane == 0) {
-    prefetch_tmap(&p.tm_q);
-    prefetch_tmap(&p.tm_z);
-    prefetch_tmap(&p.tm_y);
-  }
-  if (warp < kConsumerWarps) {
+  {
     // S of this (sequence, head) into the B tile: rows 8w .. 8w+7, 8-byte piece `lane`.
     const uint2* src = reinterpret_cast<const uint2*>(p.state + (int64_t)ch.pair * 128 * 128);
 #pragma unroll
@@ -555,19 +498,39 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
   }
   // n as the first column of the third panel: the MMA's column d is n . phi(q~).
   if (tid < 128) write_extra_row(Bs + 2 * kPanel, tid, p.norm_n[(int64_t)ch.pair * 128 + tid], false);
-  for (int i = tid; i < 4 * 128; i += kThreads) sm.w[0][i] = p.conv_q[h * 4 * 128 + i];
+  for (int i = tid; i < 4 * 128; i += kConsumers) sm.w[0][i] = p.conv_q[h * 4 * 128 + i];
   if (tid < 128) sm.gw[tid] = 0.5f * p.norm_w[h * 128 + tid];   // g / 2 (see the epilogue)
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
-
-  if (warp == kProducerWarp) {
-    const Ring rings[2] = {{{&p.tm_q, nullptr}, 1, 8, kRawPanel, kQStage, qring, sm.full[0], sm.empty[0]},
-                           {{&p.tm_z, nullptr}, 1, 0, kPanel, kZStage, zring, sm.full[1], sm.empty[1]}};
-    produce(ch, sm, rings, 2, p.status);
-  } else {
+  // No producer warp: thread 0 issues the copies.  q of tile t goes into q stage t % 2 once
+  // every warp has convolved tile t - 2 (the tile barrier of iteration t - 2); z of tile t into
+  // z stage t % 2 once the epilogue of tile t - 2 is done (the tile barrier of iteration t).
+  auto issue_q = [&](int t) {
+    const int s = t & 1, y0 = ch.seq_lo + (ch.tile0 + t) * 128;
+    mbar_expect_tx(&sm.full[0][s], kQStage);
+#pragma unroll
+    for (int pn = 0; pn < 2; ++pn)
+      tma_load_2d(qring + s * kQStage + pn * kRawPanel, &p.tm_q, h * 128 + pn * 64, y0 - 8, &sm.full[0][s]);
+  };
+  auto issue_z = [&](int t) {
+    const int s = t & 1, y0 = ch.seq_lo + (ch.tile0 + t) * 128;
+    mbar_expect_tx(&sm.full[1][s], kZStage);
+#pragma unroll
+    for (int pn = 0; pn < 2; ++pn)
+      tma_load_2d(zring + s * kZStage + pn * kPanel, &p.tm_z, h * 128 + pn * 64, y0, &sm.full[1][s]);
+  };
+  int q_issued = 0, z_issued = 0;
+  if (tid == 0) {
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_z);
+    prefetch_tmap(&p.tm_y);
+    for (; q_issued < 2 && q_issued < ch.n_tiles; ++q_issued) issue_q(q_issued);
+    for (; z_issued < 2 && z_issued < ch.n_tiles; ++z_issued) issue_z(z_issued);
+  }
+  {
     const int g = warp, c4 = lane;
     __nv_bfloat16* yx = reinterpret_cast<__nv_bfloat16*>(p.y);
     constexpr uint32_t idesc = make_idesc(128, kN, true);
@@ -641,7 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         bulk_wait_read();
         stores_pending = true;
       }
-      if (__all_sync(0xffffffffu, zok) && lane == 0) mbar_arrive(&sm.empty[1][zs]);
+      __syncwarp();
     };
 
     for (int i = 0; i < ch.n_tiles; ++i) {
@@ -655,7 +618,6 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
               phi2(x[2], x[3]);
               uq[rr] = pack4(x);
             });
-      if (__all_sync(0xffffffffu, landed) && lane == 0) mbar_arrive(&sm.empty[0][s]);
       // The previous tile's MMAs must have read A (and finished its accumulator) first.
       if (ok && i > 0) ok = wait_phase(&sm.mma_done[(i - 1) & 1], ((i - 1) >> 1) & 1, sm, p.status);
       if (ok) {
@@ -669,6 +631,16 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
         break;
       }
       if (warp == 0) {
+        if (lane == 0) {
+          if (i + 2 < ch.n_tiles) {
+            issue_q(i + 2);
+            ++q_issued;
+          }
+          if (i >= 2) {
+            issue_z(i);
+            ++z_issued;
+          }
+        }
         tc_fence_after();
         const uint64_t ad = sdesc_sw128(smem_u32(A), 16, 1024), bd = sdesc_sw128(smem_u32(Bs), kPanel, 1024);
 #pragma unroll
@@ -680,6 +652,11 @@ __global__ void __launch_bounds__(kThreads, 1) gbla_out_kernel(const __grid_cons
       }
       if (i > 0) epilogue(i - 1);
       done = i + 1;
+    }
+    if (tid == 0 && !ok) {
+      // Aborting: let the copies in flight land before the CTA releases its shared memory.
+      for (int t = (q_issued > 2 ? q_issued - 2 : 0); t < q_issued; ++t) drain_phase(&sm.full[0][t & 1], (t >> 1) & 1);
+      for (int t = (z_issued > 2 ? z_issued - 2 : 0); t < z_issued; ++t) drain_phase(&sm.full[1][t & 1], (t >> 1) & 1);
     }
     if (done > 0) {
       const int j = done - 1;
@@ -704,7 +681,7 @@ cudaError_t launch_gbla(const GblaParams& p, int n_chunks, int n_pairs, cudaStre
   if (e != cudaSuccess) return e;
   gbla_state_kernel<<<n_chunks, kConsumers, kStateSmem, s>>>(p);
   gbla_reduce_kernel<<<dim3(n_pairs, (128 * 128 + 128 + 255) / 256), 256, 0, s>>>(p);
-  gbla_out_kernel<<<n_chunks, kThreads, kOutSmem, s>>>(p);
+  gbla_out_kernel<<<n_chunks, kConsumers, kOutSmem, s>>>(p);
   return cudaGetLastError();
 }
 
