@@ -99,6 +99,7 @@ struct GblaSmem {
   float ss[4][128];                 // output: partial sums of squares of each row, per 32-column block
   uint64_t full[2][2];              // [ring][stage]: the stage's copies have landed
   uint64_t mma_done[2];             // per accumulator (the state kernel uses one)
+  float red[kConsumerWarps];        // state: per-warp maximum gate logit of the chunk
   uint64_t wait_ns;                 // bound on every wait (the launch's wait limit)
   uint32_t tmem_slot;
   int abort;
@@ -140,8 +141,6 @@ __device__ __forceinline__ void gated_phi2(float& x0, float& x1, float w, float 
   e1 = ex2(e1);
   ffma2c(x0, x1, fmaxf(x0, 0.f), fmaxf(x1, 0.f), w, w, e0, e1);
 }
-// sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation.
-__device__ __forceinline__ float sigmoidf_(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
 __device__ __forceinline__ void unpack4(const uint2& u, float (&f)[4]) {
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
@@ -329,11 +328,33 @@ __global__ void __launch_bounds__(kConsumers, 1) gbla_state_kernel(const __grid_
   // The ones column: n = sum over tokens of w phi(k~) comes out of the MMA as column d.
   if (tid < 128) write_extra_row(B + 2 * kPanel, tid, 1.f, true);
   if (warp == 0) tmem_alloc(&sm.tmem_slot, 256);
+  const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
+  {
+    // The chunk's largest gate logit (for the operand scale below).
+    const int t_lo = lo + ch.tile0 * 128, t_hi = min(hi, lo + (ch.tile0 + ch.n_tiles) * 128);
+    float amax = -INFINITY;
+    for (int t = t_lo + tid; t < t_hi; t += kConsumers) amax = fmaxf(amax, __bfloat162float(ax[(int64_t)t * H + h]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) sm.red[warp] = amax;
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_slot;
+  // Operand scale 2^es: the chunk's largest gate w_max = sigmoid(max a) times 2^es lies in
+  // (1/2, 1], so w phi(k~) keeps fp16's range whatever the gates (a chunk of nearly closed gates
+  // would otherwise underflow to 0); the partial state and n are divided by 2^es (exactly) at
+  // the end.  es = floor(-log2 w_max) = floor(log2(1 + 2^(-max a log2 e))), at most 100.
+  int es;
+  {
+    float amax = sm.red[0];
+#pragma unroll
+    for (int w = 1; w < kConsumerWarps; ++w) amax = fmaxf(amax, sm.red[w]);
+    const float l = lg2_approx(1.f + ex2(-amax * kLog2e));
+    es = l < 100.f ? (int)l : 100;
+  }
   // Tile t's k and v (two panels each, from 8 rows before the tile) into stage t % 2.
   auto issue = [&](int t) {
     const int s = t & 1, y0 = ch.seq_lo + (ch.tile0 + t) * 128;
@@ -352,7 +373,6 @@ __global__ void __launch_bounds__(kConsumers, 1) gbla_state_kernel(const __grid_
     for (; issued < 2 && issued < ch.n_tiles; ++issued) issue(issued);
   }
   const int g = warp, c4 = lane;
-  const __nv_bfloat16* ax = reinterpret_cast<const __nv_bfloat16*>(p.a);
   // fp16 operands (A and B of one type, as kind::f16 requires): the rounding of w phi(k~) and
   // v~ is the largest error of the layer (the output's RMS normalisation magnifies it in rows
   // whose weighted average nearly cancels), and fp16 has 3 more mantissa bits than bf16; both
@@ -375,8 +395,9 @@ __global__ void __launch_bounds__(kConsumers, 1) gbla_state_kernel(const __grid_
     const int first = 3 - kRowsT * g - 128 * (ch.tile0 + i);
     const float a = a_next;
     a_next = load_gate(i + 1);
-    // w = sigmoid(a), log2 w = -log2(1 + 2^(-a log2 e)); row r's pair is read from lane r.
-    const float w_l = sigmoidf_(a), lw_l = -lg2_approx(1.f + ex2(-a * kLog2e));
+    // log2 w = -log2(1 + 2^(-a log2 e)) for w = sigmoid(a), and the scaled gate 2^(log2 w + es)
+    // (exact in relative terms however small w is); row r's pair is read from lane r.
+    const float lw_l = (float)es - lg2_approx(1.f + ex2(-a * kLog2e)), w_l = ex2(lw_l);
     ok = wait_phase(&sm.full[0][s], (i >> 1) & 1, sm, p.status);
     uint2 uk[kRowsT], uv[kRowsT];
     // Both operand tiles into registers first (no wait between the two convolutions, so they
@@ -435,17 +456,18 @@ __global__ void __launch_bounds__(kConsumers, 1) gbla_state_kernel(const __grid_
     const int qd = warp & 3, cb = warp >> 2;
     const int i = 32 * qd + lane;
     const bool keep = ok && done > 0;
+    const float unscale = __int_as_float((127 - es) << 23);   // 2^-es
     float4* dst = reinterpret_cast<float4*>(part + (int64_t)i * 128 + 32 * cb);
     uint32_t r[32];
     tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * cb, r);
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      dst[e] = keep ? make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                                  __uint_as_float(r[4 * e + 3]))
+      dst[e] = keep ? make_float4(__uint_as_float(r[4 * e]) * unscale, __uint_as_float(r[4 * e + 1]) * unscale,
+                                  __uint_as_float(r[4 * e + 2]) * unscale, __uint_as_float(r[4 * e + 3]) * unscale)
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     if (cb == 0) {
       const float nv = tmem_ld1(tmem + ((uint32_t)(32 * qd) << 16) + 128);
-      part[128 * 128 + i] = keep ? nv : 0.f;
+      part[128 * 128 + i] = keep ? nv * unscale : 0.f;
     }
   }
   tc_fence_before();

@@ -84,6 +84,21 @@ def test_gbla_gate_closed_tokens_are_forgotten():
     check(y.float().cpu().numpy(), oracle_y(x, so), "closed gates")
 
 
+@pytest.mark.parametrize("shift", [-20.0, -30.0])
+def test_gbla_nearly_closed_gates_everywhere(shift):
+    """Every key gate nearly closed (logits N(shift, 2^2): w ~ 1e-9 .. 1e-13).  The gates cancel
+    between numerator and denominator (n.phi(q~) still dwarfs the 1e-6), so the output is an
+    ordinary weighted average of normal magnitude; the gated keys must not vanish in the
+    operands' range on the way."""
+    lens, H = [3000, 700], 2
+    x, so = make_inputs(lens, H, seed=31)
+    x["a"] = (x["a"].float() + shift).to(torch.bfloat16)
+    y = run_gpu(x, so, H)
+    ref = oracle_y(x, so)
+    assert np.abs(ref).max() > 1.0, "the case must have outputs of normal magnitude"
+    check(y.float().cpu().numpy(), ref, f"gates shifted by {shift}")
+
+
 def test_gbla_long_history_sampled():
     """The bench workload's shape for one sequence: a 32768-token history (H = 8), checked on
     256 sampled rows of every head."""
