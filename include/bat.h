@@ -257,6 +257,9 @@ bat_status bat_gbla_plan_chunks(const bat_gbla_plan* plan, void* dst, size_t dst
  *   workspace       device scratch of at least bat_gbla_workspace_bytes(plan) bytes
  * All device pointers 16-byte aligned (a: 2-byte).  Asynchronous on `stream`; three kernel
  * launches (state, reduce, output).  One plan and workspace run on one stream at a time.
+ * Precision: the state contraction takes w*phi(k~) (scaled per chunk by a power of two so that
+ * the chunk's largest gate is in (1/2, 1]) and v~ as fp16 operands, so |v~| and phi(k~) must stay
+ * below 65504; the output contraction takes phi(q~) and S as bf16; accumulation is fp32.
  * Errors: BAT_ERR_INVALID_ARG (null or misaligned pointer, workspace too small, host-only
  * plan, wrong device), BAT_ERR_CUDA.
  */
